@@ -1,0 +1,167 @@
+"""fp64 CPU oracle for Sparse Query Attention (test infrastructure only).
+
+Imported only by ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py``.  Nothing in the product path imports or calls it.
+
+What it restates, and from where:
+
+* Sparse Query Attention keeps the Grouped Query Attention head sharing but
+  cuts the number of *query* heads: H_q < H query heads attend, and each of
+  the H_kv key/value heads serves G = H_q / H_kv query heads.
+  ("ReactiveAI/GQA-Ref-Micro" model card, introduction;
+  "ReactiveAI/xSMQAT-m" model card, introduction;
+  "Sparse Query Attention (SQA): A Computationally Efficient Attention
+  Mechanism with Query Heads Reduction", abstract.)
+* Query and output projections shrink to width H_q * d_head.
+  ("ReactiveAI/xSMQAT-m" model card, note on model size;
+  "ReactiveAI/GQA-Ref-Micro" model card, note on model size.)
+* Causal masking for the decoder models (the training/inference usage on
+  both model cards) and no mask for encoder-style work (abstract).
+
+The pages print no equations, so the attention itself is the textbook
+definition that "extension to Grouped Query Attention" presupposes.  Readings
+taken where the pages are silent:
+
+* query head h reads key/value head j = floor(h / G) (contiguous groups);
+* scale = 1 / sqrt(d_head), passed explicitly;
+* causal: query t sees keys 0..t (diagonal included);
+* softmax in natural base, max-subtracted for range only;
+* everything in fp64 from inputs given as exact float64 copies of bf16;
+  no intermediate rounding anywhere.
+
+Evaluation proceeds one (batch, query head) pair and one chunk of query rows
+at a time.  Rows are independent in the definition, so the chunking changes
+no arithmetic of any row; it only bounds memory.  Library matmuls (numpy) are
+the only primitives used.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+_CHUNK = 256
+
+
+def _check_heads(H_q: int, H_kv: int) -> int:
+    if H_kv <= 0 or H_q <= 0 or H_q % H_kv != 0:
+        raise ValueError(f"H_q={H_q} must be a positive multiple of H_kv={H_kv}")
+    return H_q // H_kv
+
+
+def _scores(q_rows, k_head, t_rows, causal, scale):
+    """s[r, u] = scale * <q_r, k_u>, with u > t_r set to -inf when causal.
+
+    Only keys 0..max(t_rows) can be unmasked in the causal case, so the
+    columns beyond are never formed; masked entries inside are -inf.
+    """
+    if causal:
+        n_keys = int(t_rows.max()) + 1
+        k_head = k_head[:n_keys]
+    s = scale * (q_rows @ k_head.T)
+    if causal:
+        u = np.arange(k_head.shape[0])
+        s[u[None, :] > t_rows[:, None]] = -np.inf
+    return s, k_head.shape[0]
+
+
+def attention_forward(q, k, v, causal: bool, scale: float, rows=None):
+    """Sparse Query Attention output and log-sum-exp.
+
+    q: [B, N, H_q, d]; k, v: [B, N, H_kv, d] (float64 arrays).
+    rows: optional 1-D array of query token indices; all rows when None.
+    Returns o [B, R, H_q, d] and lse [B, H_q, R] (R = number of rows), with
+        o[b,t,h]   = sum_u softmax_u(s_tu) v[b,u,j],  j = h // G
+        lse[b,h,t] = log sum_u exp(s_tu)
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, N, H_q, d = q.shape
+    H_kv = k.shape[2]
+    G = _check_heads(H_q, H_kv)
+    t_all = np.arange(N) if rows is None else np.asarray(rows, dtype=np.int64)
+    R = t_all.shape[0]
+    o = np.empty((B, R, H_q, d), dtype=np.float64)
+    lse = np.empty((B, H_q, R), dtype=np.float64)
+    for b in range(B):
+        for h in range(H_q):
+            j = h // G
+            for c0 in range(0, R, _CHUNK):
+                t = t_all[c0:c0 + _CHUNK]
+                s, n_keys = _scores(q[b, t, h, :], k[b, :, j, :], t, causal, scale)
+                m = s.max(axis=1, keepdims=True)
+                w = np.exp(s - m)
+                l = w.sum(axis=1)
+                o[b, c0:c0 + len(t), h, :] = (w @ v[b, :n_keys, j, :]) / l[:, None]
+                lse[b, h, c0:c0 + len(t)] = m[:, 0] + np.log(l)
+    return o, lse
+
+
+def attention_backward(q, k, v, do, causal: bool, scale: float):
+    """Gradients of L = sum(o * do) with respect to q, k and v.
+
+    Chain rule through the definition above, per (b, h) with j = h // G:
+        P   = softmax rows of s
+        dP  = do_h v_j^T
+        dS  = P * (dP - rowsum(P * dP))      (softmax Jacobian)
+        dq_h  = scale * dS k_j
+        dk_j += scale * dS^T q_h             (summed over the G heads of group j)
+        dv_j += P^T do_h                     (summed over the G heads of group j)
+    Returns dq [B,N,H_q,d], dk and dv [B,N,H_kv,d].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    B, N, H_q, d = q.shape
+    H_kv = k.shape[2]
+    G = _check_heads(H_q, H_kv)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    t_all = np.arange(N)
+    for b in range(B):
+        for h in range(H_q):
+            j = h // G
+            for c0 in range(0, N, _CHUNK):
+                t = t_all[c0:c0 + _CHUNK]
+                s, n_keys = _scores(q[b, t, h, :], k[b, :, j, :], t, causal, scale)
+                m = s.max(axis=1, keepdims=True)
+                w = np.exp(s - m)
+                p = w / w.sum(axis=1, keepdims=True)
+                g = do[b, t, h, :]
+                dp = g @ v[b, :n_keys, j, :].T
+                ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
+                dq[b, t, h, :] = scale * (ds @ k[b, :n_keys, j, :])
+                dk[b, :n_keys, j, :] += scale * (ds.T @ q[b, t, h, :])
+                dv[b, :n_keys, j, :] += p.T @ g
+    return dq, dk, dv
+
+
+def projection(x, w, bias=None):
+    """y = x w^T (+ bias): x [M, K], w [Nout, K] in nn.Linear layout."""
+    y = np.asarray(x, dtype=np.float64) @ np.asarray(w, dtype=np.float64).T
+    if bias is not None:
+        y = y + np.asarray(bias, dtype=np.float64)[None, :]
+    return y
+
+
+def sqa_layer_forward(x, wq, wk, wv, wo, B: int, N: int, H_q: int, H_kv: int,
+                      d_head: int, causal: bool = True, scale=None):
+    """One SQA attention layer: reduced-width Q/K/V projections, the
+    attention core, and the output projection from H_q*d_head back to
+    d_model.  All in fp64 with no intermediate rounding.
+
+    x [B*N, d_model]; wq [H_q*d, d_model]; wk, wv [H_kv*d, d_model];
+    wo [d_model, H_q*d].  Returns a dict with q, k, v, o (attention output,
+    [B*N, H_q*d]) and y [B*N, d_model].
+    """
+    if scale is None:
+        scale = 1.0 / np.sqrt(d_head)
+    q = projection(x, wq).reshape(B, N, H_q, d_head)
+    k = projection(x, wk).reshape(B, N, H_kv, d_head)
+    v = projection(x, wv).reshape(B, N, H_kv, d_head)
+    o, lse = attention_forward(q, k, v, causal, scale)
+    o2 = o.reshape(B * N, H_q * d_head)
+    y = projection(o2, wo)
+    return {"q": q, "k": k, "v": v, "o": o2, "lse": lse, "y": y}

@@ -1,0 +1,360 @@
+"""Pins for the fp64 oracle, independent of the oracle's own code (CPU only).
+
+Each check ties the oracle to something other than itself: hand-derived
+closed forms (tests/golden), a pure-Python brute force with a different
+evaluation order (unstabilised softmax, math.fsum), a library routine
+(torch scaled_dot_product_attention and autograd in fp64), finite
+differences, invariants of softmax attention, and the closed-form FLOP count
+behind the query-head reduction ("Sparse Query Attention (SQA): A
+Computationally Efficient Attention Mechanism with Query Heads Reduction",
+abstract: attention FLOPs fall in proportion to the number of query heads).
+"""
+
+import itertools
+import json
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from oracle import attention_backward, attention_forward, projection, sqa_layer_forward
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "closed_form_cases.json")
+
+
+# ----------------------------------------------------------------------------
+# Independent brute force: nested Python loops, unstabilised softmax, fsum.
+# It also counts the multiply-adds of the two contractions it performs.
+# ----------------------------------------------------------------------------
+class _Counter:
+    def __init__(self):
+        self.qk = 0
+        self.pv = 0
+
+
+def brute_attention(q, k, v, causal, scale, counter=None):
+    B, N, H_q, d = q.shape
+    H_kv = k.shape[2]
+    G = H_q // H_kv
+    o = np.zeros((B, N, H_q, d))
+    lse = np.zeros((B, H_q, N))
+    for b in range(B):
+        for h in range(H_q):
+            j = h // G
+            for t in range(N):
+                keys = range(t + 1) if causal else range(N)
+                e = []
+                for u in keys:
+                    s = scale * math.fsum(float(q[b, t, h, c]) * float(k[b, u, j, c]) for c in range(d))
+                    if counter is not None:
+                        counter.qk += d
+                    e.append(math.exp(s))
+                z = math.fsum(e)
+                for c in range(d):
+                    o[b, t, h, c] = math.fsum(e[i] * float(v[b, u, j, c]) for i, u in enumerate(keys)) / z
+                    if counter is not None:
+                        counter.pv += len(e)
+                lse[b, h, t] = math.log(z)
+    return o, lse
+
+
+def _rand(shape, rng, scale=1.0):
+    return rng.standard_normal(shape) * scale
+
+
+def _expand(x):
+    """Numbers, or the fixture's small expressions in ln3 / ln4."""
+    if isinstance(x, str):
+        expr = re.sub(r"(\d)(ln[34])", r"\1*\2", x)
+        return float(eval(expr, {"__builtins__": {}}, {"ln3": math.log(3.0), "ln4": math.log(4.0)}))
+    return float(x)
+
+
+def _arr(nested):
+    def walk(x):
+        return [walk(y) for y in x] if isinstance(x, list) else _expand(x)
+    return np.array(walk(nested), dtype=np.float64)
+
+
+# ----------------------------------------------------------------------------
+# Closed forms worked by hand
+# ----------------------------------------------------------------------------
+def _golden_cases():
+    with open(GOLDEN) as f:
+        return json.load(f)["cases"]
+
+
+@pytest.mark.parametrize("case", _golden_cases(), ids=lambda c: c["name"])
+def test_closed_form_cases(case):
+    q = _arr(case["q"])[None]
+    k = _arr(case["k"])[None]
+    v = _arr(case["v"])[None]
+    o, lse = attention_forward(q, k, v, case["causal"], case["scale"])
+    np.testing.assert_allclose(o[0], _arr(case["o"]), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse[0], _arr(case["lse"]), rtol=1e-15, atol=1e-12)
+    if "dq" in case:
+        dq, dk, dv = attention_backward(q, k, v, _arr(case["do"])[None], case["causal"], case["scale"])
+        np.testing.assert_allclose(dq[0], _arr(case["dq"]), atol=1e-12)
+        np.testing.assert_allclose(dk[0], _arr(case["dk"]), atol=1e-12)
+        np.testing.assert_allclose(dv[0], _arr(case["dv"]), atol=1e-12)
+
+
+def test_golden_expander():
+    assert _expand("-1.5ln3") == pytest.approx(-1.5 * math.log(3))
+    assert _expand("1+ln3/1000") == pytest.approx(1 + math.log(3) / 1000)
+    assert _expand("1000+ln4") == pytest.approx(1000 + math.log(4))
+
+
+# ----------------------------------------------------------------------------
+# Brute force on tiny inputs
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("heads", [(1, 1), (2, 1), (2, 2), (4, 2), (4, 1)])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N,d", [(1, 1), (3, 2), (6, 4)])
+def test_brute_force_tiny(heads, causal, N, d):
+    H_q, H_kv = heads
+    rng = np.random.default_rng(N * 100 + d * 10 + H_q + causal)
+    B = 2
+    q = _rand((B, N, H_q, d), rng)
+    k = _rand((B, N, H_kv, d), rng)
+    v = _rand((B, N, H_kv, d), rng)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = attention_forward(q, k, v, causal, scale)
+    ob, lseb = brute_attention(q, k, v, causal, scale)
+    np.testing.assert_allclose(o, ob, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lseb, rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# Reduction to standard attention: torch SDPA (fp64, CPU) as a library check
+# ----------------------------------------------------------------------------
+def _sdpa(q, k, v, causal, scale, gqa):
+    tq = torch.from_numpy(q).permute(0, 2, 1, 3)
+    tk = torch.from_numpy(k).permute(0, 2, 1, 3)
+    tv = torch.from_numpy(v).permute(0, 2, 1, 3)
+    o = F.scaled_dot_product_attention(tq, tk, tv, is_causal=causal, scale=scale, enable_gqa=gqa)
+    return o.permute(0, 2, 1, 3).numpy()
+
+
+@pytest.mark.parametrize("heads", [(4, 4), (8, 4), (8, 2), (4, 1), (16, 4)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_matches_sdpa(heads, causal):
+    H_q, H_kv = heads
+    rng = np.random.default_rng(7 + H_q * 3 + H_kv + causal)
+    B, N, d = 2, 37, 16
+    q, k, v = _rand((B, N, H_q, d), rng), _rand((B, N, H_kv, d), rng), _rand((B, N, H_kv, d), rng)
+    scale = 1.0 / math.sqrt(d)
+    o, _ = attention_forward(q, k, v, causal, scale)
+    np.testing.assert_allclose(o, _sdpa(q, k, v, causal, scale, H_q != H_kv), rtol=0, atol=1e-12)
+
+
+def test_gqa_expansion_identity():
+    """SQA(H_q, H_kv) equals MHA with H_q heads on K/V repeated G times
+    (contiguous groups); gradients of K/V are the group sums of the MHA ones."""
+    rng = np.random.default_rng(11)
+    B, N, H_q, H_kv, d = 2, 19, 8, 2, 8
+    G = H_q // H_kv
+    q, k, v = _rand((B, N, H_q, d), rng), _rand((B, N, H_kv, d), rng), _rand((B, N, H_kv, d), rng)
+    do = _rand((B, N, H_q, d), rng)
+    kr, vr = np.repeat(k, G, axis=2), np.repeat(v, G, axis=2)
+    for causal in (False, True):
+        o, lse = attention_forward(q, k, v, causal, 0.3)
+        o2, lse2 = attention_forward(q, kr, vr, causal, 0.3)
+        np.testing.assert_allclose(o, o2, atol=1e-13)
+        np.testing.assert_allclose(lse, lse2, atol=1e-13)
+        dq, dk, dv = attention_backward(q, k, v, do, causal, 0.3)
+        dq2, dk2, dv2 = attention_backward(q, kr, vr, do, causal, 0.3)
+        np.testing.assert_allclose(dq, dq2, atol=1e-12)
+        np.testing.assert_allclose(dk, dk2.reshape(B, N, H_kv, G, d).sum(3), atol=1e-12)
+        np.testing.assert_allclose(dv, dv2.reshape(B, N, H_kv, G, d).sum(3), atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# Softmax and attention invariants
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("causal", [False, True])
+def test_rows_sum_to_one_and_mask_is_zero(causal):
+    """With d = N and V the identity (v[u] = e_u), o[t] is the probability
+    row itself: it sums to 1, and masked entries are exactly 0."""
+    rng = np.random.default_rng(3)
+    B, N, H_q, H_kv = 1, 12, 4, 2
+    q = _rand((B, N, H_q, N), rng)
+    k = _rand((B, N, H_kv, N), rng)
+    v = np.broadcast_to(np.eye(N)[None, :, None, :], (B, N, H_kv, N)).copy()
+    o, _ = attention_forward(q, k, v, causal, 0.5)
+    np.testing.assert_allclose(o.sum(axis=-1), 1.0, atol=1e-12)
+    assert (o >= 0).all()
+    if causal:
+        upper = np.triu(np.ones((N, N), dtype=bool), 1)
+        assert (o[0][:, 0][upper] == 0).all()
+        assert (o[0].transpose(1, 0, 2)[:, upper] == 0).all()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_identical_keys_give_mean_of_v(causal):
+    rng = np.random.default_rng(5)
+    B, N, H_q, H_kv, d = 2, 9, 4, 2, 3
+    q = _rand((B, N, H_q, d), rng)
+    k = np.broadcast_to(_rand((B, 1, H_kv, d), rng), (B, N, H_kv, d)).copy()
+    v = _rand((B, N, H_kv, d), rng)
+    do = _rand((B, N, H_q, d), rng)
+    o, _ = attention_forward(q, k, v, causal, 0.7)
+    G = H_q // H_kv
+    for t in range(N):
+        keys = slice(0, t + 1) if causal else slice(0, N)
+        for h in range(H_q):
+            np.testing.assert_allclose(o[:, t, h], v[:, keys, h // G].mean(axis=1), atol=1e-13)
+    dq, _, _ = attention_backward(q, k, v, do, causal, 0.7)
+    np.testing.assert_allclose(dq, 0.0, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gradient_invariants(causal):
+    """sum_u dS_tu = 0 gives sum_u dk[u] = 0 per kv head; and
+    sum_u dv[u, j] = sum over the group's heads and all t of do."""
+    rng = np.random.default_rng(8)
+    B, N, H_q, H_kv, d = 2, 14, 6, 2, 5
+    q, k, v = _rand((B, N, H_q, d), rng), _rand((B, N, H_kv, d), rng), _rand((B, N, H_kv, d), rng)
+    do = _rand((B, N, H_q, d), rng)
+    dq, dk, dv = attention_backward(q, k, v, do, causal, 0.4)
+    np.testing.assert_allclose(dk.sum(axis=1), 0.0, atol=1e-12)
+    G = H_q // H_kv
+    want = do.reshape(B, N, H_kv, G, d).sum(axis=(1, 3))
+    np.testing.assert_allclose(dv.sum(axis=1), want, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# Gradients: central differences of the brute force, and torch autograd
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_finite_differences(causal):
+    rng = np.random.default_rng(21 + causal)
+    B, N, H_q, H_kv, d = 1, 4, 2, 1, 3
+    q, k, v = _rand((B, N, H_q, d), rng), _rand((B, N, H_kv, d), rng), _rand((B, N, H_kv, d), rng)
+    do = _rand((B, N, H_q, d), rng)
+    scale = 0.6
+    dq, dk, dv = attention_backward(q, k, v, do, causal, scale)
+    eps = 1e-6
+
+    def loss(q_, k_, v_):
+        o, _ = brute_attention(q_, k_, v_, causal, scale)
+        return math.fsum((o * do).ravel())
+
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        fd = np.zeros_like(x)
+        for idx in itertools.product(*[range(n) for n in x.shape]):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = {"q": q, "k": k, "v": v}
+            args_m = {"q": q, "k": k, "v": v}
+            args_p[name], args_m[name] = xp, xm
+            fd[idx] = (loss(**{a + "_": b for a, b in args_p.items()})
+                       - loss(**{a + "_": b for a, b in args_m.items()})) / (2 * eps)
+        err = np.abs(fd - g).max() / max(np.abs(g).max(), 1e-300)
+        assert err < 1e-6, (name, err)
+
+
+@pytest.mark.parametrize("heads", [(4, 4), (8, 4), (4, 1)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_matches_autograd(heads, causal):
+    H_q, H_kv = heads
+    rng = np.random.default_rng(31 + H_q + H_kv + causal)
+    B, N, d = 2, 23, 8
+    q, k, v = _rand((B, N, H_q, d), rng), _rand((B, N, H_kv, d), rng), _rand((B, N, H_kv, d), rng)
+    do = _rand((B, N, H_q, d), rng)
+    scale = 1 / math.sqrt(d)
+    tq, tk, tv = (torch.from_numpy(a.copy()).permute(0, 2, 1, 3).requires_grad_() for a in (q, k, v))
+    o = F.scaled_dot_product_attention(tq, tk, tv, is_causal=causal, scale=scale, enable_gqa=H_q != H_kv)
+    o.backward(torch.from_numpy(do).permute(0, 2, 1, 3))
+    dq, dk, dv = attention_backward(q, k, v, do, causal, scale)
+    np.testing.assert_allclose(dq, tq.grad.permute(0, 2, 1, 3).numpy(), atol=1e-12)
+    np.testing.assert_allclose(dk, tk.grad.permute(0, 2, 1, 3).numpy(), atol=1e-12)
+    np.testing.assert_allclose(dv, tv.grad.permute(0, 2, 1, 3).numpy(), atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# Sampled rows, chunk boundaries
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("causal", [False, True])
+def test_sampled_rows_equal_full_rows(causal):
+    rng = np.random.default_rng(13)
+    B, N, H_q, H_kv, d = 1, 600, 4, 2, 8   # N spans several 256-row chunks
+    q, k, v = _rand((B, N, H_q, d), rng), _rand((B, N, H_kv, d), rng), _rand((B, N, H_kv, d), rng)
+    o, lse = attention_forward(q, k, v, causal, 0.35)
+    rows = np.array([0, 1, 255, 256, 257, 511, 512, 599])
+    os_, lses = attention_forward(q, k, v, causal, 0.35, rows=rows)
+    np.testing.assert_allclose(os_, o[:, rows], atol=1e-13)
+    np.testing.assert_allclose(lses, lse[:, :, rows], atol=1e-13)
+    ob, lseb = brute_attention(q[:, :40], k[:, :40], v[:, :40], causal, 0.35) if causal else (None, None)
+    if causal:  # causal rows < 40 only see the first 40 keys
+        np.testing.assert_allclose(o[:, :40], ob, atol=1e-12)
+        np.testing.assert_allclose(lse[:, :, :40], lseb, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# FLOP accounting: the query-head reduction factor
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("causal", [False, True])
+def test_flop_count_scales_with_query_heads(causal):
+    """The brute force's counted multiply-adds per contraction equal
+    B * H_q * P_c * d (P_c = N(N+1)/2 causal, N^2 otherwise), so MHA / SQA
+    costs H / H_q exactly, independent of H_kv."""
+    B, N, d, H = 1, 7, 2, 8
+    counts = {}
+    for H_q, H_kv in ((8, 8), (8, 2), (4, 4), (4, 1), (2, 2)):
+        rng = np.random.default_rng(0)
+        c = _Counter()
+        brute_attention(_rand((B, N, H_q, d), rng), _rand((B, N, H_kv, d), rng),
+                        _rand((B, N, H_kv, d), rng), causal, 1.0, counter=c)
+        P_c = N * (N + 1) // 2 if causal else N * N
+        assert c.qk == B * H_q * P_c * d
+        assert c.pv == B * H_q * P_c * d
+        counts[(H_q, H_kv)] = c.qk + c.pv
+    assert counts[(8, 8)] == counts[(8, 2)]
+    for (H_q, H_kv), n in counts.items():
+        assert counts[(H, H)] * H_q == n * H
+
+
+# ----------------------------------------------------------------------------
+# Projections and the layer
+# ----------------------------------------------------------------------------
+def test_projection_naive_loop_and_matmul():
+    rng = np.random.default_rng(17)
+    M, K, Nout = 5, 7, 3
+    x, w, bias = _rand((M, K), rng), _rand((Nout, K), rng), _rand((Nout,), rng)
+    y = projection(x, w, bias)
+    for m in range(M):
+        for n in range(Nout):
+            assert y[m, n] == pytest.approx(math.fsum(x[m, c] * w[n, c] for c in range(K)) + bias[n], abs=1e-13)
+    big_x, big_w = _rand((64, 48), rng), _rand((40, 48), rng)
+    ref = torch.from_numpy(big_x) @ torch.from_numpy(big_w).T
+    np.testing.assert_allclose(projection(big_x, big_w), ref.numpy(), atol=1e-12)
+
+
+def test_layer_against_torch_composition():
+    """The layer equals nn.functional.linear -> SDPA (GQA) -> linear in fp64."""
+    rng = np.random.default_rng(19)
+    B, N, d_model, H_q, H_kv, dh = 2, 17, 32, 4, 2, 8
+    x = _rand((B * N, d_model), rng)
+    wq, wk, wv = _rand((H_q * dh, d_model), rng, .1), _rand((H_kv * dh, d_model), rng, .1), _rand((H_kv * dh, d_model), rng, .1)
+    wo = _rand((d_model, H_q * dh), rng, .1)
+    out = sqa_layer_forward(x, wq, wk, wv, wo, B, N, H_q, H_kv, dh, causal=True)
+    tx = torch.from_numpy(x)
+    tq = F.linear(tx, torch.from_numpy(wq)).view(B, N, H_q, dh).transpose(1, 2)
+    tk = F.linear(tx, torch.from_numpy(wk)).view(B, N, H_kv, dh).transpose(1, 2)
+    tv = F.linear(tx, torch.from_numpy(wv)).view(B, N, H_kv, dh).transpose(1, 2)
+    to = F.scaled_dot_product_attention(tq, tk, tv, is_causal=True, enable_gqa=True)
+    ty = F.linear(to.transpose(1, 2).reshape(B * N, H_q * dh), torch.from_numpy(wo))
+    np.testing.assert_allclose(out["y"], ty.numpy(), atol=1e-12)
+
+
+def test_rejects_bad_head_counts():
+    q = np.zeros((1, 2, 3, 4))
+    k = np.zeros((1, 2, 2, 4))
+    with pytest.raises(ValueError):
+        attention_forward(q, k, k, False, 1.0)
