@@ -1,0 +1,344 @@
+"""Throughput of the Sparse Query Attention core on B200.
+
+One step = one forward pass of the SQA attention core over the encoder-style
+long-sequence workload: B=1, N=32768 tokens, d_head=128, non-causal, SQA head
+counts H_q=8 query heads sharing H_kv=4 key/value heads (of H=16 head slots),
+bf16 Q/K/V ~ N(0,1), fp32 output [B, N, H_q*d_head], through sqa_attn_fwd.
+The same kernel at H_q=H=16 (MHA) and the other head-count variants are timed
+beside it to give the speed-up that the query-head reduction buys.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sqa|reference]
+
+Prints ONE JSON line on rank 0.  Multi-GPU runs (torchrun, one rank per GPU)
+give every rank its own independent problem of the same size (weak scaling,
+no data-path collective); time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = {"workload": "sqa_encoder_fwd_32k", "B": 1, "N": 32768, "H_q": 8, "H_kv": 4, "H": 16,
+            "d_head": 128, "causal": False, "out": "fp32"}
+VARIANTS = {"MHA": (16, 16), "GQA": (16, 4), "SQA": (8, 4), "sSQA": (8, 8), "xSQA": (4, 4)}
+METRIC = "SQA attention TFLOP/s and tokens/s at 32k-200k tokens; % of B200 BF16 peak"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def attn_fwd_flops(B, N, H_q, d, causal):
+    """Algorithmic FLOPs of the core forward: two contractions of
+    2 * B * H_q * P_c * d each, P_c the unmasked (query, key) pairs."""
+    P_c = N * (N + 1) // 2 if causal else N * N
+    return 4 * B * H_q * P_c * d
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p.get("bf16_tflops", 1590.0), "measured"
+    return 1590.0, "fallback"
+
+
+def csrc_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "sparse_query_attention_b200", "csrc")
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(d, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic():
+    """DRAM bytes per launch of the forward kernel from the committed ncu
+    summary, valid only while the kernel sources are unchanged."""
+    path = os.path.join(ROOT, "profiles", "sqa_fwd_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    if t.get("csrc_sha") != csrc_hash() or t.get("workload") != WORKLOAD["workload"]:
+        return None
+    return t.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# CPU baseline: the oracle as it stands, on a bounded sample of the workload.
+# ----------------------------------------------------------------------------
+def cpu_baseline(rows_per_head=128, seed=2):
+    import numpy as np
+    import torch
+    from oracle import attention_forward
+    from sqa_inputs import attention_inputs, sample_rows
+
+    w = WORKLOAD
+    x = attention_inputs(w["B"], w["N"], w["H_q"], w["H_kv"], w["d_head"], seed, device="cpu")
+    q, k, v = (t.double().numpy() for t in (x["q"], x["k"], x["v"]))
+    rows = sample_rows(w["N"], rows_per_head, seed)
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:  # noqa: BLE001
+        cores = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    attention_forward(q, k, v, w["causal"], 1 / math.sqrt(w["d_head"]), rows=rows)
+    dt = time.perf_counter() - t0
+    flops = 4 * w["B"] * w["H_q"] * len(rows) * w["N"] * w["d_head"]
+    del np, torch
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": int(cores), "kind": "oracle",
+            "sample": f"{len(rows)} query rows x {w['H_q']} heads of the N={w['N']} workload "
+                      f"({flops / 1e9:.1f} GFLOP, {dt:.2f} s, fp64 numpy)",
+            "seconds": dt, "tokens_per_s": w["B"] * len(rows) / dt}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    per_step = []
+    base = None
+    for i in range(args.warmup + args.steps):
+        b = cpu_baseline(rows_per_head=16 if args.steps > 3 else 32)
+        if i >= args.warmup:
+            per_step.append(b)
+        base = b
+    secs = sum(b["seconds"] for b in per_step)
+    flops = sum(b["value"] * b["seconds"] * 1e12 for b in per_step)
+    val = flops / secs / 1e12
+    line = {"metric": METRIC, "value": val, "unit": "TFLOP/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / len(per_step),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": dict(WORKLOAD, sample=base["sample"]),
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": base["cores"], "kind": "oracle",
+                             "sample": base["sample"]},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+def run_sqa(args):
+    import torch
+    import torch.distributed as dist
+
+    import sparse_query_attention_b200 as sqa
+    from sqa_inputs import attention_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    w = WORKLOAD
+    B, N, H_q, H_kv, d = w["B"], w["N"], w["H_q"], w["H_kv"], w["d_head"]
+    scale = 1 / math.sqrt(d)
+    flops_step = attn_fwd_flops(B, N, H_q, d, w["causal"])
+
+    x = attention_inputs(B, N, H_q, H_kv, d, seed=2 + rank, device=dev)
+    out = torch.empty((B, N, H_q * d), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(q, k, v, o, h_q=H_q, h_kv=H_kv):
+        sqa.sqa_attn_fwd(q, k, v, o, B, N, h_q, h_kv, d, w["causal"], scale, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(val):
+        if world == 1:
+            return val
+        t = torch.tensor([val], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step(x["q"], x["k"], x["v"], out)
+    sqa.sqa_device_status(stream)
+
+    # --- timed region: K steps, L2 flushed between steps (not timed) -------
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            starts[i].record(stream)
+            step(x["q"], x["k"], x["v"], out)
+            ends[i].record(stream)
+        barrier()
+    sqa.sqa_device_status(stream)
+    per_launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = max_over_ranks(sum(per_launch_ms))
+    ms_per_step = total_ms / args.steps
+    value = world * flops_step * args.steps / (total_ms / 1e3) / 1e12
+    tokens_per_s = world * B * N * args.steps / (total_ms / 1e3)
+
+    # --- end to end through the C ABI with host buffers --------------------
+    hq, hk, hv = (t.cpu().pin_memory() for t in (x["q"], x["k"], x["v"]))
+    ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dq_, dk_, dv_ = (torch.empty_like(t) for t in (x["q"], x["k"], x["v"]))
+    e2e_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        for hsrc, ddst in ((hq, dq_), (hk, dk_), (hv, dv_)):
+            ddst.copy_(hsrc, non_blocking=True)
+        step(dq_, dk_, dv_, out)
+        ho.copy_(out, non_blocking=True)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for hsrc, ddst in ((hq, dq_), (hk, dk_), (hv, dv_)):
+            ddst.copy_(hsrc, non_blocking=True)
+        step(dq_, dk_, dv_, out)
+        ho.copy_(out, non_blocking=True)
+    e1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_value = world * flops_step * e2e_steps / (e2e_ms / 1e3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size()
+
+    # --- head-count variants on the same kernel (speed-up vs H_q = H) ------
+    variants = {}
+    for name, (vq, vkv) in VARIANTS.items():
+        xv = attention_inputs(B, N, vq, vkv, d, seed=2, device=dev)
+        ov = torch.empty((B, N, vq * d), dtype=torch.float32, device=dev)
+        for _ in range(2):
+            step(xv["q"], xv["k"], xv["v"], ov, vq, vkv)
+        times = []
+        for _ in range(5):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            step(xv["q"], xv["k"], xv["v"], ov, vq, vkv)
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        ms = statistics.median(times)
+        variants[name] = {"H_q": vq, "H_kv": vkv, "ms": ms,
+                          "tflops": attn_fwd_flops(B, N, vq, d, w["causal"]) / (ms / 1e3) / 1e12}
+        del xv, ov
+    for name in variants:
+        variants[name]["speedup_vs_mha"] = variants["MHA"]["ms"] / variants[name]["ms"]
+        variants[name]["ideal_speedup"] = VARIANTS["MHA"][0] / variants[name]["H_q"]
+    sqa.sqa_device_status(stream)
+
+    peak, peak_kind = load_peaks()
+    achieved = flops_step / (statistics.mean(per_launch_ms) / 1e3) / 1e12
+    traffic = load_traffic()
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(WORKLOAD, parallelism=f"independent problems x{world}",
+                       l2="flushed between timed steps (256 MiB write)"),
+        "tokens_per_s": tokens_per_s,
+        "pct_of_bf16_peak": 100 * achieved / peak,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic, "peak_source": f"{peak_kind} bf16 burst"},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "variants": variants,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = {k: v for k, v in cpu_baseline().items() if k not in ("seconds",)}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["sqa", "reference"], default="sqa")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_sqa(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

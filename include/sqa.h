@@ -1,0 +1,136 @@
+/*
+ * sqa.h - C ABI of the Sparse Query Attention hot path for NVIDIA B200 (sm_100a).
+ *
+ * Sparse Query Attention keeps the key/value sharing of Grouped Query
+ * Attention but lowers the number of *query* heads: H_q query heads attend,
+ * and each of the H_kv key/value heads is shared by G = H_q / H_kv
+ * consecutive query heads (query head h reads key/value head h / G).  Score
+ * and context FLOPs therefore scale with H_q instead of the full head count H.
+ *   - "ReactiveAI/GQA-Ref-Micro" model card, introduction (SQA as an
+ *     extension of GQA that reduces query heads);
+ *   - "Sparse Query Attention (SQA): A Computationally Efficient Attention
+ *     Mechanism with Query Heads Reduction", abstract (FLOPs fall in
+ *     proportion to the query-head reduction; pre-training, fine-tuning and
+ *     encoder workloads; 32k-200k token sequences);
+ *   - "ReactiveAI/xSMQAT-m" model card, note on model size (query and output
+ *     projections shrink to width H_q * d_head).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *    library allocates no device memory and keeps no per-call state.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL means the legacy default stream).  Nothing synchronises except
+ *    sqa_device_status().
+ *  - Layouts are dense, row-major, with the last index contiguous:
+ *      Q, O, dO, dQ : [B, N, H_q,  d_head]
+ *      K, V, dK, dV : [B, N, H_kv, d_head]
+ *      LSE          : [B, H_q, N]  (fp32, natural log of the softmax sum)
+ *    so O viewed as [B*N, H_q*d_head] is the input of the output projection.
+ *  - Tensor pointers must be 16-byte aligned.
+ *  - Invalid arguments return SQA_ERR_INVALID_ARG and launch nothing; shapes
+ *    the kernels do not handle return SQA_ERR_UNSUPPORTED; a failed launch
+ *    returns SQA_ERR_CUDA.
+ *  - Device-side waits are bounded.  A wait that runs out records
+ *    SQA_ERR_TIMEOUT in a device status word (the kernel then winds down and
+ *    returns); sqa_device_status() reports and clears it.
+ */
+#ifndef SQA_H_
+#define SQA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SQA_OK = 0,
+  SQA_ERR_INVALID_ARG = 1,
+  SQA_ERR_UNSUPPORTED = 2,
+  SQA_ERR_CUDA = 3,
+  SQA_ERR_TIMEOUT = 4
+} sqa_status_t;
+
+typedef enum { SQA_DT_F32 = 0, SQA_DT_BF16 = 1 } sqa_dtype_t;
+
+/*
+ * sqa_attn_fwd - attention core forward, fp32 output.
+ *   O[b,t,h,:] = sum_u softmax_u(scale * <Q[b,t,h,:], K[b,u,j,:]>) V[b,u,j,:],
+ *   j = h / (H_q / H_kv); with causal != 0 only keys u <= t take part.
+ * q, k, v : bf16, layouts above.   out : fp32 [B, N, H_q * d_head].
+ * Requirements: B, N >= 1; 1 <= H_kv <= H_q; H_q % H_kv == 0;
+ * d_head in {16, 32, 64, 128} (else SQA_ERR_UNSUPPORTED); scale finite.
+ */
+sqa_status_t sqa_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                          int B, int N, int H_q, int H_kv, int d_head, int causal,
+                          float scale, void* stream);
+
+/*
+ * sqa_attn_fwd_ex - as sqa_attn_fwd, with the output dtype chosen by
+ * out_dtype (SQA_DT_F32 or SQA_DT_BF16) and, when lse != NULL, the
+ * per-row log-sum-exp of the scaled scores written to lse [B, H_q, N] fp32
+ * (natural log; what sqa_attn_bwd needs).
+ */
+sqa_status_t sqa_attn_fwd_ex(const void* q, const void* k, const void* v, void* out,
+                             sqa_dtype_t out_dtype, float* lse,
+                             int B, int N, int H_q, int H_kv, int d_head, int causal,
+                             float scale, void* stream);
+
+/*
+ * sqa_attn_bwd_workspace_size - bytes of device workspace sqa_attn_bwd needs
+ * for this shape (the per-row dot products D = rowsum(dO * O), fp32).
+ * Returns 0 for invalid shapes.
+ */
+size_t sqa_attn_bwd_workspace_size(int B, int N, int H_q, int H_kv, int d_head);
+
+/*
+ * sqa_attn_bwd - gradient of the attention core (the training step the
+ * pages' throughput claims are about).
+ * Inputs : q, k, v (bf16), out = the forward output O (dtype o_dtype),
+ *          dout = dL/dO (bf16, [B,N,H_q,d_head]),
+ *          lse  = the forward's log-sum-exp [B,H_q,N] fp32.
+ * Outputs: dq [B,N,H_q,d], dk and dv [B,N,H_kv,d] in grad_dtype (F32 or
+ *          BF16).  dk and dv of key/value head j are summed over the G query
+ *          heads of group j.  All three are fully overwritten.
+ * workspace: device buffer of at least sqa_attn_bwd_workspace_size() bytes,
+ *          owned by the caller, 16-byte aligned; contents on entry ignored.
+ */
+sqa_status_t sqa_attn_bwd(const void* q, const void* k, const void* v,
+                          const void* out, sqa_dtype_t o_dtype,
+                          const void* dout, const float* lse,
+                          void* dq, void* dk, void* dv, sqa_dtype_t grad_dtype,
+                          int B, int N, int H_q, int H_kv, int d_head, int causal,
+                          float scale, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/*
+ * sqa_proj - one reduced-width projection, Y[M, Nout] = X[M, K] W[Nout, K]^T
+ * (+ bias), the Q/K/V projections (Nout = H_q*d_head or H_kv*d_head) and the
+ * output projection (K = H_q*d_head).  X and W are bf16 (W in nn.Linear
+ * layout); bias is NULL or fp32 [Nout]; Y is y_dtype (F32 or BF16).
+ * Requirements: M, K, Nout >= 1; K % 16 == 0; Nout % 16 == 0.
+ */
+sqa_status_t sqa_proj(const void* x, const void* w, const float* bias, void* y,
+                      sqa_dtype_t y_dtype, int M, int K, int Nout, void* stream);
+
+/*
+ * sqa_device_status - synchronises `stream`, then returns SQA_ERR_TIMEOUT if
+ * any kernel of this library on the current device gave up a bounded wait
+ * since the last call (and clears the record), SQA_ERR_CUDA if the stream
+ * reports an error, else SQA_OK.
+ */
+sqa_status_t sqa_device_status(void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* sqa_status_string(sqa_status_t status);
+
+/* Library version, "major.minor.patch". */
+const char* sqa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQA_H_ */

@@ -1,0 +1,139 @@
+"""Python binding of libsqa.so, the B200 (sm_100a) Sparse Query Attention hot path.
+
+Each function has the name and argument order of the C entry point in
+``include/sqa.h`` and only marshals arguments: tensors become raw device
+pointers, ``stream=None`` becomes torch's current CUDA stream, and a non-OK
+status raises :class:`SQAError`.  Every step of the computation runs in the
+library's CUDA kernels; there is no other implementation behind these names.
+
+The library must have been built (``python -m sparse_query_attention_b200.build``);
+importing this package without it raises ImportError.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+from .build import LIB_PATH
+
+SQA_OK = 0
+SQA_ERR_INVALID_ARG = 1
+SQA_ERR_UNSUPPORTED = 2
+SQA_ERR_CUDA = 3
+SQA_ERR_TIMEOUT = 4
+
+SQA_DT_F32 = 0
+SQA_DT_BF16 = 1
+
+# Every symbol include/sqa.h declares, with (restype, argtypes).
+_P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "sqa_attn_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "sqa_attn_fwd_ex": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "sqa_attn_bwd_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
+    "sqa_attn_bwd": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I,
+                          _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
+    "sqa_proj": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "sqa_device_status": (_I, [_P]),
+    "sqa_status_string": (ctypes.c_char_p, [_I]),
+    "sqa_version": (ctypes.c_char_p, []),
+}
+
+
+class SQAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing; build it with `python -m sparse_query_attention_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+def _ptr(x):
+    """Device pointer of a CUDA tensor (or an int / None passed through)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if not x.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not x.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str) -> None:
+    if status != SQA_OK:
+        raise SQAError(status, where)
+
+
+def status_string(status: int) -> str:
+    return _lib.sqa_status_string(int(status)).decode()
+
+
+def sqa_version() -> str:
+    return _lib.sqa_version().decode()
+
+
+def sqa_status_string(status: int) -> str:
+    return status_string(status)
+
+
+def sqa_attn_fwd(q, k, v, out, B, N, H_q, H_kv, d_head, causal, scale, stream=None) -> None:
+    _check(_lib.sqa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, N, H_q, H_kv, d_head,
+                             int(bool(causal)), float(scale), _stream(stream)), "sqa_attn_fwd")
+
+
+def sqa_attn_fwd_ex(q, k, v, out, out_dtype, lse, B, N, H_q, H_kv, d_head, causal, scale,
+                    stream=None) -> None:
+    _check(_lib.sqa_attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(out_dtype), _ptr(lse),
+                                B, N, H_q, H_kv, d_head, int(bool(causal)), float(scale),
+                                _stream(stream)), "sqa_attn_fwd_ex")
+
+
+def sqa_attn_bwd_workspace_size(B, N, H_q, H_kv, d_head) -> int:
+    return int(_lib.sqa_attn_bwd_workspace_size(B, N, H_q, H_kv, d_head))
+
+
+def sqa_attn_bwd(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B, N, H_q, H_kv,
+                 d_head, causal, scale, workspace, workspace_bytes, stream=None) -> None:
+    _check(_lib.sqa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(o_dtype), _ptr(dout),
+                             _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), int(grad_dtype),
+                             B, N, H_q, H_kv, d_head, int(bool(causal)), float(scale),
+                             _ptr(workspace), int(workspace_bytes), _stream(stream)),
+           "sqa_attn_bwd")
+
+
+def sqa_proj(x, w, bias, y, y_dtype, M, K, Nout, stream=None) -> None:
+    _check(_lib.sqa_proj(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), int(y_dtype), M, K, Nout,
+                         _stream(stream)), "sqa_proj")
+
+
+def sqa_device_status(stream=None) -> None:
+    _check(_lib.sqa_device_status(_stream(stream)), "sqa_device_status")

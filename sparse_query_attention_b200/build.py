@@ -1,0 +1,84 @@
+"""Builds libsqa.so (the C ABI in include/sqa.h) in-tree with nvcc for sm_100a.
+
+    python -m sparse_query_attention_b200.build [--force] [--verbose]
+"""
+
+from __future__ import annotations
+
+import argparse
+import os
+import shutil
+import subprocess
+import sys
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG_DIR)
+CSRC = os.path.join(PKG_DIR, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+LIB_PATH = os.path.join(PKG_DIR, "libsqa.so")
+MAIN_SOURCE = os.path.join(CSRC, "sqa_api.cu")
+
+ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def _nvcc() -> str:
+    for cand in (shutil.which("nvcc"), "/usr/local/cuda/bin/nvcc"):
+        if cand and os.path.exists(cand):
+            return cand
+    raise RuntimeError("nvcc not found: the SQA CUDA library cannot be built")
+
+
+def _sources():
+    out = [os.path.join(INCLUDE, "sqa.h")]
+    for name in sorted(os.listdir(CSRC)):
+        if name.endswith((".cu", ".cuh")):
+            out.append(os.path.join(CSRC, name))
+    return out
+
+
+def is_stale() -> bool:
+    if not os.path.exists(LIB_PATH):
+        return True
+    built = os.path.getmtime(LIB_PATH)
+    return any(os.path.getmtime(p) > built for p in _sources())
+
+
+def nvcc_command(extra=()):
+    return [
+        _nvcc(), *ARCH_FLAGS, "-O3", "-lineinfo", "-std=c++17",
+        "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr",
+        "-I", INCLUDE, "-I", CSRC,
+        *extra,
+        "-o", LIB_PATH, MAIN_SOURCE,
+    ]
+
+
+def build(force: bool = False, verbose: bool = False, extra=()) -> str:
+    """Compile libsqa.so if missing or older than its sources; returns its path."""
+    if not force and not is_stale():
+        return LIB_PATH
+    cmd = nvcc_command(extra)
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
+    if verbose and (res.stdout or res.stderr):
+        print(res.stdout, res.stderr, sep="\n", flush=True)
+    return LIB_PATH
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--ptxas-info", action="store_true", help="print register/smem use per kernel")
+    args = ap.parse_args(argv)
+    extra = ["-Xptxas", "-v"] if args.ptxas_info else []
+    build(force=args.force or args.ptxas_info, verbose=args.verbose or args.ptxas_info, extra=extra)
+    print(LIB_PATH)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,267 @@
+// sqa_api.cu - the C ABI declared in include/sqa.h: argument checks, TMA
+// tensor-map encoding, kernel selection and launch.  One translation unit so
+// the device status word and every kernel live in the same module.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "sqa.h"
+#include "sqa_attn_simt.cuh"
+#include "sqa_proj_kernel.cuh"
+#include "sqa_ptx.cuh"
+
+namespace {
+
+using sqa::kProjBM;
+
+// ---------------------------------------------------------------------------
+// Driver entry point for cuTensorMapEncodeTiled, fetched once through the
+// runtime (no link-time dependency on libcuda).
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool encode_fn_ready() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// A bf16 tensor map of rank `rank`; dims/strides innermost first, strides in
+// bytes for dims 1.., box in elements, 128-byte swizzle unless given.
+bool make_map_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                   const uint64_t* strides_bytes, const uint32_t* box,
+                   CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+  if (!encode_fn_ready()) return false;
+  cuuint32_t elem_strides[5] = {1, 1, 1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base),
+                        reinterpret_cast<const cuuint64_t*>(dims), reinterpret_cast<const cuuint64_t*>(strides_bytes),
+                        reinterpret_cast<const cuuint32_t*>(box), elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+sqa_status_t launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
+}
+
+bool supported_d(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+sqa_status_t check_attn_args(const void* q, const void* k, const void* v, int B, int N, int H_q, int H_kv, int d,
+                             float scale) {
+  if (!q || !k || !v) return SQA_ERR_INVALID_ARG;
+  if (B <= 0 || N <= 0 || H_q <= 0 || H_kv <= 0 || H_kv > H_q || H_q % H_kv != 0) return SQA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return SQA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return SQA_ERR_INVALID_ARG;
+  if (d <= 0) return SQA_ERR_INVALID_ARG;
+  if (!supported_d(d)) return SQA_ERR_UNSUPPORTED;
+  // Row indices are formed in 32-bit arithmetic inside the kernels.
+  if (static_cast<long long>(B) * N * H_q > (1ll << 31) - 1) return SQA_ERR_UNSUPPORTED;
+  return SQA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Attention forward
+// ---------------------------------------------------------------------------
+template <int D>
+void launch_fwd_simt(const void* q, const void* k, const void* v, void* out, int out_bf16, float* lse, int B, int N,
+                     int H_q, int H_kv, int causal, float scale, cudaStream_t st) {
+  dim3 grid((N + sqa::kSimtRows - 1) / sqa::kSimtRows, H_q, B);
+  sqa::attn_fwd_simt_kernel<D><<<grid, sqa::kSimtRows, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+      static_cast<const __nv_bfloat16*>(v), out, out_bf16, lse, N, H_q, H_kv, causal, scale);
+}
+
+sqa_status_t attn_fwd_impl(const void* q, const void* k, const void* v, void* out, sqa_dtype_t out_dtype, float* lse,
+                           int B, int N, int H_q, int H_kv, int d, int causal, float scale, void* stream) {
+  sqa_status_t s = check_attn_args(q, k, v, B, N, H_q, H_kv, d, scale);
+  if (s != SQA_OK) return s;
+  if (!out || !aligned16(out) || (lse && !aligned16(lse))) return SQA_ERR_INVALID_ARG;
+  if (out_dtype != SQA_DT_F32 && out_dtype != SQA_DT_BF16) return SQA_ERR_INVALID_ARG;
+  const int ob = out_dtype == SQA_DT_BF16;
+  cudaStream_t st = as_stream(stream);
+  switch (d) {
+    case 16: launch_fwd_simt<16>(q, k, v, out, ob, lse, B, N, H_q, H_kv, causal, scale, st); break;
+    case 32: launch_fwd_simt<32>(q, k, v, out, ob, lse, B, N, H_q, H_kv, causal, scale, st); break;
+    case 64: launch_fwd_simt<64>(q, k, v, out, ob, lse, B, N, H_q, H_kv, causal, scale, st); break;
+    default: launch_fwd_simt<128>(q, k, v, out, ob, lse, B, N, H_q, H_kv, causal, scale, st); break;
+  }
+  return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// Attention backward
+// ---------------------------------------------------------------------------
+size_t bwd_workspace_bytes(int B, int N, int H_q) {
+  const size_t rows = static_cast<size_t>(B) * H_q * N;
+  return ((rows * sizeof(float)) + 255) & ~size_t(255);
+}
+
+template <int D, typename GradT>
+void launch_bwd_simt(const void* q, const void* k, const void* v, const void* o, int o_bf16, const void* dout,
+                     const float* lse, void* dq, void* dk, void* dv, int B, int N, int H_q, int H_kv, int causal,
+                     float scale, float* dsum, cudaStream_t st) {
+  const auto* qb = static_cast<const __nv_bfloat16*>(q);
+  const auto* kb = static_cast<const __nv_bfloat16*>(k);
+  const auto* vb = static_cast<const __nv_bfloat16*>(v);
+  const auto* gb = static_cast<const __nv_bfloat16*>(dout);
+  const size_t rows = static_cast<size_t>(B) * N * H_q;
+  const unsigned dot_blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
+  sqa::attn_bwd_dot_kernel<D><<<dot_blocks, 256, 0, st>>>(o, o_bf16, gb, dsum, B, N, H_q);
+  dim3 gq((N + sqa::kSimtRows - 1) / sqa::kSimtRows, H_q, B);
+  sqa::attn_bwd_dq_simt_kernel<D, GradT><<<gq, sqa::kSimtRows, 0, st>>>(qb, kb, vb, gb, lse, dsum,
+                                                                          static_cast<GradT*>(dq), N, H_q, H_kv,
+                                                                          causal, scale);
+  dim3 gk((N + sqa::kSimtRows - 1) / sqa::kSimtRows, H_kv, B);
+  sqa::attn_bwd_dkdv_simt_kernel<D, GradT><<<gk, sqa::kSimtRows, 0, st>>>(
+      qb, kb, vb, gb, lse, dsum, static_cast<GradT*>(dk), static_cast<GradT*>(dv), N, H_q, H_kv, causal, scale);
+}
+
+template <int D>
+void launch_bwd_d(bool grad_bf16, const void* q, const void* k, const void* v, const void* o, int o_bf16,
+                  const void* dout, const float* lse, void* dq, void* dk, void* dv, int B, int N, int H_q, int H_kv,
+                  int causal, float scale, float* dsum, cudaStream_t st) {
+  if (grad_bf16)
+    launch_bwd_simt<D, __nv_bfloat16>(q, k, v, o, o_bf16, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale,
+                                      dsum, st);
+  else
+    launch_bwd_simt<D, float>(q, k, v, o, o_bf16, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, dsum, st);
+}
+
+// ---------------------------------------------------------------------------
+// Projection GEMM
+// ---------------------------------------------------------------------------
+template <int BN, bool kBf16>
+sqa_status_t launch_proj_bn(const CUtensorMap& mx, const CUtensorMap& mw, const float* bias, void* y, int M, int K,
+                            int Nout, cudaStream_t st) {
+  auto kern = sqa::proj_gemm_kernel<BN, kBf16>;
+  constexpr int smem = sqa::ProjSmem<BN>::kDynamicBytes;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return SQA_ERR_CUDA;
+  dim3 grid((M + kProjBM - 1) / kProjBM, (Nout + BN - 1) / BN);
+  kern<<<grid, 128, smem, st>>>(mx, mw, bias, y, M, K, Nout);
+  return launch_status();
+}
+
+template <bool kBf16>
+sqa_status_t launch_proj(const CUtensorMap& mx, const void* w, const float* bias, void* y, int M, int K, int Nout,
+                         cudaStream_t st) {
+  // BN: the narrowest tile that covers Nout, at most 256.
+  int bn = 16;
+  while (bn < Nout && bn < 256) bn *= 2;
+  CUtensorMap mw;
+  const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(Nout)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(K) * 2};
+  const uint32_t box[2] = {64, static_cast<uint32_t>(bn)};
+  if (!make_map_bf16(&mw, w, 2, dims, strides, box)) return SQA_ERR_CUDA;
+  switch (bn) {
+    case 16: return launch_proj_bn<16, kBf16>(mx, mw, bias, y, M, K, Nout, st);
+    case 32: return launch_proj_bn<32, kBf16>(mx, mw, bias, y, M, K, Nout, st);
+    case 64: return launch_proj_bn<64, kBf16>(mx, mw, bias, y, M, K, Nout, st);
+    case 128: return launch_proj_bn<128, kBf16>(mx, mw, bias, y, M, K, Nout, st);
+    default: return launch_proj_bn<256, kBf16>(mx, mw, bias, y, M, K, Nout, st);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+sqa_status_t sqa_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int N, int H_q, int H_kv,
+                          int d_head, int causal, float scale, void* stream) {
+  return attn_fwd_impl(q, k, v, out, SQA_DT_F32, nullptr, B, N, H_q, H_kv, d_head, causal, scale, stream);
+}
+
+sqa_status_t sqa_attn_fwd_ex(const void* q, const void* k, const void* v, void* out, sqa_dtype_t out_dtype,
+                             float* lse, int B, int N, int H_q, int H_kv, int d_head, int causal, float scale,
+                             void* stream) {
+  return attn_fwd_impl(q, k, v, out, out_dtype, lse, B, N, H_q, H_kv, d_head, causal, scale, stream);
+}
+
+size_t sqa_attn_bwd_workspace_size(int B, int N, int H_q, int H_kv, int d_head) {
+  if (B <= 0 || N <= 0 || H_q <= 0 || H_kv <= 0 || H_kv > H_q || H_q % H_kv != 0 || d_head <= 0) return 0;
+  return bwd_workspace_bytes(B, N, H_q);
+}
+
+sqa_status_t sqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, sqa_dtype_t o_dtype,
+                          const void* dout, const float* lse, void* dq, void* dk, void* dv, sqa_dtype_t grad_dtype,
+                          int B, int N, int H_q, int H_kv, int d_head, int causal, float scale, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  sqa_status_t s = check_attn_args(q, k, v, B, N, H_q, H_kv, d_head, scale);
+  if (s != SQA_OK) return s;
+  if (!out || !dout || !lse || !dq || !dk || !dv || !workspace) return SQA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(dout) || !aligned16(lse) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv) || !aligned16(workspace))
+    return SQA_ERR_INVALID_ARG;
+  if ((o_dtype != SQA_DT_F32 && o_dtype != SQA_DT_BF16) || (grad_dtype != SQA_DT_F32 && grad_dtype != SQA_DT_BF16))
+    return SQA_ERR_INVALID_ARG;
+  if (workspace_bytes < bwd_workspace_bytes(B, N, H_q)) return SQA_ERR_INVALID_ARG;
+  float* dsum = static_cast<float*>(workspace);
+  const bool gb = grad_dtype == SQA_DT_BF16;
+  const int ob = o_dtype == SQA_DT_BF16;
+  cudaStream_t st = as_stream(stream);
+  switch (d_head) {
+    case 16: launch_bwd_d<16>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, dsum, st); break;
+    case 32: launch_bwd_d<32>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, dsum, st); break;
+    case 64: launch_bwd_d<64>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, dsum, st); break;
+    default: launch_bwd_d<128>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, dsum, st); break;
+  }
+  return launch_status();
+}
+
+sqa_status_t sqa_proj(const void* x, const void* w, const float* bias, void* y, sqa_dtype_t y_dtype, int M, int K,
+                      int Nout, void* stream) {
+  if (!x || !w || !y) return SQA_ERR_INVALID_ARG;
+  if (M <= 0 || K <= 0 || Nout <= 0) return SQA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y) || (bias && !aligned16(bias))) return SQA_ERR_INVALID_ARG;
+  if (y_dtype != SQA_DT_F32 && y_dtype != SQA_DT_BF16) return SQA_ERR_INVALID_ARG;
+  if (K % 16 != 0 || Nout % 16 != 0) return SQA_ERR_UNSUPPORTED;
+  CUtensorMap mx;
+  const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(K) * 2};
+  const uint32_t box[2] = {64, static_cast<uint32_t>(kProjBM)};
+  if (!make_map_bf16(&mx, x, 2, dims, strides, box)) return SQA_ERR_CUDA;
+  cudaStream_t st = as_stream(stream);
+  return y_dtype == SQA_DT_BF16 ? launch_proj<true>(mx, w, bias, y, M, K, Nout, st)
+                                : launch_proj<false>(mx, w, bias, y, M, K, Nout, st);
+}
+
+sqa_status_t sqa_device_status(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return SQA_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, sqa::g_status_word, sizeof(word)) != cudaSuccess) return SQA_ERR_CUDA;
+  if (word != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(sqa::g_status_word, &zero, sizeof(zero)) != cudaSuccess) return SQA_ERR_CUDA;
+    return SQA_ERR_TIMEOUT;
+  }
+  return SQA_OK;
+}
+
+const char* sqa_status_string(sqa_status_t status) {
+  switch (status) {
+    case SQA_OK: return "SQA_OK";
+    case SQA_ERR_INVALID_ARG: return "SQA_ERR_INVALID_ARG";
+    case SQA_ERR_UNSUPPORTED: return "SQA_ERR_UNSUPPORTED";
+    case SQA_ERR_CUDA: return "SQA_ERR_CUDA";
+    case SQA_ERR_TIMEOUT: return "SQA_ERR_TIMEOUT";
+  }
+  return "SQA_ERR_UNKNOWN";
+}
+
+const char* sqa_version(void) { return "0.1.0"; }
+
+}  // extern "C"

@@ -1,0 +1,380 @@
+// sqa_fwd_kernel.cuh - fused Sparse Query Attention forward on sm_100a.
+//
+// What it computes (per batch b, query head h, query token t; j = h / G,
+// G = H_q / H_kv):
+//   O[b,t,h,:] = sum_u softmax_u(scale * <Q[b,t,h,:], K[b,u,j,:]>) V[b,u,j,:]
+//   LSE[b,h,t] = log sum_u exp(scale * <Q[b,t,h,:], K[b,u,j,:]>)
+// with u <= t when causal.  Only H_q query heads exist, so the two
+// contractions cost 2 * B * H_q * P_c * d FLOPs each: the query-head
+// reduction of "Sparse Query Attention (SQA): A Computationally Efficient
+// Attention Mechanism with Query Heads Reduction" (abstract), built on the
+// key/value sharing of Grouped Query Attention ("ReactiveAI/GQA-Ref-Micro"
+// model card, introduction).
+//
+// Layout of the work.  One CTA owns two 128-row query tiles of ONE key/value
+// head j.  A tile packs g query heads of the group side by side: row
+// r = tt * g + gg is token t0 + tt, head h0 + gg (g = largest power of two
+// dividing G, at most 128; 128 / g tokens per tile).  Every K/V tile is
+// therefore fetched once by TMA and used by all the query heads the CTA
+// holds -- the GQA/SQA sharing turned into on-chip reuse.
+//
+// Roles (12 warps):
+//   warp 0 (one lane)  TMA: Q tiles once, then K_i, V_i into a ring of slots.
+//   warp 1 (one lane)  tcgen05.mma issue:  S_t = Q_t K_i^T  (SMEM x SMEM ->
+//                      TMEM fp32), O_t += P_t V_i (P from TMEM, V from SMEM).
+//   warps 4-7, 8-11    softmax for tile 0 / tile 1, one thread per row:
+//                      TMEM S -> registers, mask, online max/sum in the log2
+//                      domain, P = 2^(s - m) as bf16 back into TMEM over S,
+//                      rescale of O in TMEM when the running max grew by more
+//                      than 2^8, and the epilogue O / l, LSE.
+// TMEM (512 columns): S_0 | S_1 | O_0 | O_1  (128, 128, d, d columns); P_t
+// occupies the first 64 columns of S_t.
+// MMA order per KV step i: PV_0(i), S_0(i+1), PV_1(i), S_1(i+1), so that the
+// softmax of one tile overlaps the tensor-core work of the other.
+#pragma once
+
+#include "sqa_ptx.cuh"
+
+namespace sqa {
+
+template <int D>
+struct FwdCfg {
+  static_assert(D == 16 || D == 32 || D == 64 || D == 128, "head dim");
+  static constexpr int kRowElems = D < 64 ? D : 64;  // elements per swizzled smem row
+  static constexpr int kRowBytes = kRowElems * 2;    // 32, 64 or 128
+  static constexpr int kChunks = D / kRowElems;      // 64-wide column chunks (1 or 2)
+  static constexpr int kChunkBytes = 128 * kRowBytes;
+  static constexpr int kTileBytes = kChunks * kChunkBytes;  // one 128 x D bf16 tile
+  static constexpr uint32_t kSwizzle = kRowBytes == 128 ? kSw128 : (kRowBytes == 64 ? kSw64 : kSw32);
+  static constexpr int kSlots = D == 128 ? 4 : 6;  // K/V ring entries
+  static constexpr int kQBytes = 2 * kTileBytes;
+  static constexpr int kSmemBytes = kQBytes + kSlots * kTileBytes + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
+};
+
+struct FwdParams {
+  void* out;       // [B, N, H_q, D], fp32 or bf16
+  float* lse;      // [B, H_q, N] or null
+  int B, N, H_q, H_kv, G, g, log2g;
+  int n_sub;       // G / g head sub-groups per KV head
+  int n_tblk;      // token blocks of 2 * (128 / g) tokens
+  int causal;
+  int out_bf16;
+  float scale_log2;  // scale * log2(e)
+};
+
+constexpr int kFwdThreads = 384;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only past 2^8 growth
+
+template <int D>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    sqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t q_full;
+  __shared__ __align__(8) uint64_t slot_full[C::kSlots];
+  __shared__ __align__(8) uint64_t slot_empty[C::kSlots];
+  __shared__ __align__(8) uint64_t s_full[2];
+  __shared__ __align__(8) uint64_t p_ready[2];
+  __shared__ __align__(8) uint64_t o_done[2];
+  __shared__ __align__(8) uint64_t mma_done;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_smem = smem;                   // [2][chunks][128 rows][row bytes]
+  uint8_t* ring = smem + C::kQBytes;        // [slots][chunks][128 rows][row bytes]
+
+  const int warp = warp_id_uniform();
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit -----------------------------------------------------------
+  const int T = 128 >> p.log2g;  // tokens per tile
+  const int tblk = p.causal ? (p.n_tblk - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
+  const int j = blockIdx.y / p.n_sub;
+  const int sub = blockIdx.y % p.n_sub;
+  const int b = blockIdx.z;
+  const int h0 = j * p.G + sub * p.g;
+  const int t0 = tblk * 2 * T;  // tile 0 tokens [t0, t0+T), tile 1 [t0+T, t0+2T)
+  const int n_kv_all = (p.N + 127) / 128;
+  int n_kv[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int last_tok = min(t0 + (t + 1) * T, p.N) - 1;
+    n_kv[t] = p.causal ? (last_tok < 0 ? 0 : last_tok / 128 + 1) : n_kv_all;
+  }
+  // A tile entirely past N still runs one (masked) step so its barriers stay
+  // in lock-step; its rows are never stored.
+  n_kv[0] = max(n_kv[0], 1);
+  n_kv[1] = max(n_kv[1], 1);
+  const int n_steps = max(n_kv[0], n_kv[1]);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&q_full, 1);
+    for (int s = 0; s < C::kSlots; ++s) {
+      mbar_init(&slot_full[s], 1);
+      mbar_init(&slot_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_ready[t], 4);  // one arrival per softmax warp
+      mbar_init(&o_done[t], 1);
+    }
+    mbar_init(&mma_done, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(&tmem_base_sh, C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 0) {
+    // ======================= TMA producer =================================
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&q_full, C::kQBytes);
+      for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_4d(&tm_q, &q_full, q_smem + (t * C::kChunks + c) * C::kChunkBytes, c * C::kRowElems, h0,
+                      t0 + t * T, b);
+      int load = 0;  // ring position: K_0, V_0, K_1, V_1, ...
+      bool ok = true;
+      for (int i = 0; i < n_steps && ok; ++i) {
+        for (int kv = 0; kv < 2; ++kv, ++load) {
+          const int s = load % C::kSlots;
+          if (load >= C::kSlots && !mbar_wait(&slot_empty[s], ((load / C::kSlots) - 1) & 1, &abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&slot_full[s], C::kTileBytes);
+          uint8_t* dst = ring + s * C::kTileBytes;
+          const CUtensorMap* m = kv == 0 ? &tm_k : &tm_v;
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_4d(m, &slot_full[s], dst + c * C::kChunkBytes, c * C::kRowElems, j, i * 128, b);
+        }
+      }
+      // Teardown: nothing may still be landing in shared memory at exit.
+      mbar_drain(&q_full, 0);
+      for (int l = max(0, load - C::kSlots); l < load; ++l) mbar_drain(&slot_full[l % C::kSlots], (l / C::kSlots) & 1);
+    }
+  } else if (warp == 1) {
+    // ======================= MMA issuer ===================================
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t q_addr = smem_addr(q_smem);
+      const uint32_t ring_addr = smem_addr(ring);
+      const uint32_t col_s[2] = {C::kColS0, C::kColS1};
+      const uint32_t col_o[2] = {C::kColO0, C::kColO1};
+
+      auto issue_s = [&](int t, int slot) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int c = (kk * 16) / C::kRowElems;
+          const uint32_t off = c * C::kChunkBytes + ((kk * 16) % C::kRowElems) * 2;
+          const uint64_t a = smem_desc(q_addr + t * C::kTileBytes + off, 16, 8 * C::kRowBytes, C::kSwizzle);
+          const uint64_t bd = smem_desc(ring_addr + slot * C::kTileBytes + off, 16, 8 * C::kRowBytes, C::kSwizzle);
+          mma_ss(tmem + col_s[t], a, bd, idesc_s, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int t, int slot, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // 16 keys per MMA
+          const uint64_t bd = smem_desc(ring_addr + slot * C::kTileBytes + kk * 16 * C::kRowBytes, C::kChunkBytes,
+                                        8 * C::kRowBytes, C::kSwizzle);
+          mma_ts(tmem + col_o[t], tmem + col_s[t] + kk * 8, bd, idesc_o, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+
+      bool ok = mbar_wait(&q_full, 0, &abort_flag);
+      // Step 0 scores.
+      int kslot = 0;  // ring position of K_i is 2i, of V_i is 2i + 1
+      if (ok) ok = mbar_wait(&slot_full[0], 0, &abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        mma_commit(&s_full[0]);
+        issue_s(1, 0);
+        mma_commit(&s_full[1]);
+        mma_commit(&slot_empty[0]);
+      }
+      for (int i = 0; i < n_steps && ok; ++i) {
+        const int vpos = 2 * i + 1, kpos = 2 * i + 2;
+        const int vs = vpos % C::kSlots, ks = kpos % C::kSlots;
+        if (!mbar_wait(&slot_full[vs], (vpos / C::kSlots) & 1, &abort_flag)) break;
+        const bool more = i + 1 < n_steps;
+        if (more && !mbar_wait(&slot_full[ks], (kpos / C::kSlots) & 1, &abort_flag)) break;
+        // tile 0: O_0 += P_0 V_i, then S_0 = Q_0 K_{i+1}^T
+        if (!mbar_wait(&p_ready[0], i & 1, &abort_flag)) break;
+        tc_fence_after();
+        issue_pv(0, vs, i > 0);
+        mma_commit(&o_done[0]);
+        if (more) {
+          issue_s(0, ks);
+          mma_commit(&s_full[0]);
+        }
+        // tile 1
+        if (!mbar_wait(&p_ready[1], i & 1, &abort_flag)) break;
+        tc_fence_after();
+        issue_pv(1, vs, i > 0);
+        mma_commit(&o_done[1]);
+        mma_commit(&slot_empty[vs]);
+        if (more) {
+          issue_s(1, ks);
+          mma_commit(&s_full[1]);
+          mma_commit(&slot_empty[ks]);
+        }
+      }
+      (void)kslot;
+      mma_commit(&mma_done);
+    }
+  } else if (warp >= 4) {
+    // ======================= softmax + epilogue ===========================
+    const int t = (warp - 4) >> 2;  // tile
+    const int wq = warp & 3;        // TMEM lane quarter
+    const int r = wq * 32 + lane;   // row within the tile
+    const int tok = t0 + t * T + (r >> p.log2g);
+    const int head = h0 + (r & (p.g - 1));
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const uint32_t s_addr = lane_base + (t == 0 ? C::kColS0 : C::kColS1);
+    const uint32_t o_addr = lane_base + (t == 0 ? C::kColO0 : C::kColO1);
+    const float sl2 = p.scale_log2;
+    const int tile_tok_min = t0 + t * T;
+    const int my_steps = n_steps;  // both tiles step in lock-step with the MMA warp
+
+    float m_used = -INFINITY;  // running max in log2 units (of scaled scores)
+    float l_sum = 0.f;
+    bool ok = true;
+    for (int i = 0; i < my_steps; ++i) {
+      if (!mbar_wait(&s_full[t], i & 1, &abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[128];
+      tmem_ld32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+      tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+      tmem_wait_ld();
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]) * sl2;
+      // Masking: keys past N, and keys after the query token when causal.
+      const int key0 = i * 128;
+      const bool need_mask = (key0 + 128 > p.N) || (p.causal && key0 + 127 > tile_tok_min) || i >= n_kv[t];
+      if (need_mask) {
+        int lim = p.N - key0;                                   // keys [0, lim) are < N
+        if (p.causal) lim = min(lim, tok - key0 + 1);           // keys <= tok
+        if (i >= n_kv[t]) lim = 0;
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= lim) s[c] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+      const float m_new = fmaxf(m_used, mx);
+      // Rescale only when the running max grew by more than the threshold
+      // (or on the first finite max); otherwise keep exponentiating against
+      // the stale max, which bounds P by 2^8.
+      const bool grow = m_new > m_used + kRescaleThreshold || (m_used == -INFINITY && m_new != -INFINITY);
+      if (__any_sync(0xffffffffu, grow && i > 0 && m_used != -INFINITY)) {
+        // O holds sum over steps < i; it is final once PV(i-1) completed.
+        if (!mbar_wait(&o_done[t], (i - 1) & 1, &abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float f = (grow && m_used != -INFINITY) ? ex2_approx(m_used - m_new) : 1.f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 16) {
+          uint32_t orr[16];
+          tmem_ld16(o_addr + c0, orr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * f);
+          tmem_st16(o_addr + c0, orr);
+        }
+        tmem_wait_st();
+      }
+      if (grow) {
+        l_sum *= (m_used == -INFINITY) ? 0.f : ex2_approx(m_used - m_new);
+        m_used = m_new;
+      }
+      const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
+      float rs = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float p0 = ex2_approx(s[2 * c] - m_sub);
+        const float p1 = ex2_approx(s[2 * c + 1] - m_sub);
+        rs += p0 + p1;
+        pk[c] = pack_bf16x2(p0, p1);
+      }
+      l_sum += rs;
+      tmem_st32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_ready[t]);
+    }
+    // Epilogue: O / l and LSE once the last PV of this tile has landed.
+    if (ok) ok = mbar_wait(&o_done[t], (my_steps - 1) & 1, &abort_flag);
+    if (ok) {
+      tc_fence_after();
+      const bool valid = tok < p.N;
+      const float inv_l = 1.f / l_sum;
+      const size_t row_off = ((static_cast<size_t>(b) * p.N + (valid ? tok : 0)) * p.H_q + head) * D;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 16) {
+        uint32_t orr[16];
+        tmem_ld16(o_addr + c0, orr);
+        tmem_wait_ld();
+        if (valid) {
+          float v[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) v[c] = __uint_as_float(orr[c]) * inv_l;
+          if (p.out_bf16) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + row_off + c0);
+            dst[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                                pack_bf16x2(v[6], v[7]));
+            dst[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
+                                pack_bf16x2(v[14], v[15]));
+          } else {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row_off + c0);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+              dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+          }
+        }
+      }
+      if (valid && p.lse != nullptr)
+        p.lse[(static_cast<size_t>(b) * p.H_q + head) * p.N + tok] = (m_used + __log2f(l_sum)) * 0.69314718055994531f;
+    }
+  }
+
+  // ---- teardown ------------------------------------------------------------
+  __syncwarp();
+  if (threadIdx.x == 32) mbar_drain(&mma_done, 0);  // every issued MMA has finished
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace sqa

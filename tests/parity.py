@@ -1,0 +1,63 @@
+"""Shared helpers for the GPU parity tests: the tolerance and the calls that
+run the CUDA path through the C ABI on seeded inputs."""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+# bf16 inputs, fp32 accumulation: max |err| <= 2e-2 and relative L2 error
+# <= 1e-2, per output tensor.
+ATOL = 2e-2
+RTOL_L2 = 1e-2
+
+
+def errors(got, want):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    diff = got - want
+    max_abs = float(np.abs(diff).max()) if diff.size else 0.0
+    norm = float(np.linalg.norm(want.ravel()))
+    rel_l2 = float(np.linalg.norm(diff.ravel()) / norm) if norm > 0 else float(np.linalg.norm(diff.ravel()))
+    return max_abs, rel_l2
+
+
+def assert_close(got, want, what=""):
+    got = np.asarray(got, dtype=np.float64)
+    assert np.isfinite(got).all(), f"{what}: non-finite values"
+    max_abs, rel_l2 = errors(got, want)
+    assert max_abs <= ATOL and rel_l2 <= RTOL_L2, f"{what}: max|err|={max_abs:.3e} relL2={rel_l2:.3e}"
+    return max_abs, rel_l2
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def run_fwd(sqa, q, k, v, causal, scale=None, out_dtype=torch.float32, with_lse=True):
+    """Runs sqa_attn_fwd_ex on device tensors; returns (o [B,N,H_q,d], lse)."""
+    B, N, H_q, d = q.shape
+    H_kv = k.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    out = torch.empty((B, N, H_q, d), dtype=out_dtype, device=q.device)
+    lse = torch.empty((B, H_q, N), dtype=torch.float32, device=q.device) if with_lse else None
+    dt = sqa.SQA_DT_BF16 if out_dtype == torch.bfloat16 else sqa.SQA_DT_F32
+    sqa.sqa_attn_fwd_ex(q, k, v, out, dt, lse, B, N, H_q, H_kv, d, causal, scale)
+    return out, lse
+
+
+def run_bwd(sqa, q, k, v, o, do, lse, causal, scale=None, grad_dtype=torch.float32):
+    B, N, H_q, d = q.shape
+    H_kv = k.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    dq = torch.empty_like(q, dtype=grad_dtype)
+    dk = torch.empty_like(k, dtype=grad_dtype)
+    dv = torch.empty_like(v, dtype=grad_dtype)
+    wsb = sqa.sqa_attn_bwd_workspace_size(B, N, H_q, H_kv, d)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=q.device)
+    od = sqa.SQA_DT_BF16 if o.dtype == torch.bfloat16 else sqa.SQA_DT_F32
+    gd = sqa.SQA_DT_BF16 if grad_dtype == torch.bfloat16 else sqa.SQA_DT_F32
+    sqa.sqa_attn_bwd(q, k, v, o, od, do, lse, dq, dk, dv, gd, B, N, H_q, H_kv, d, causal, scale, ws, wsb)
+    return dq, dk, dv

@@ -1,0 +1,56 @@
+"""GPU parity of the SQA attention-core gradient against the fp64 oracle."""
+
+import math
+
+import pytest
+import torch
+
+from oracle import attention_backward
+from parity import assert_close, f64, run_bwd, run_fwd
+from sqa_inputs import attention_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def sqa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import sparse_query_attention_b200 as lib
+    return lib
+
+
+def _check_bwd(sqa, B, N, H_q, H_kv, d, causal, seed, o_dtype=torch.float32, grad_dtype=torch.float32):
+    x = attention_inputs(B, N, H_q, H_kv, d, seed, with_dout=True, device="cuda")
+    o, lse = run_fwd(sqa, x["q"], x["k"], x["v"], causal, out_dtype=o_dtype)
+    dq, dk, dv = run_bwd(sqa, x["q"], x["k"], x["v"], o, x["do"], lse, causal, grad_dtype=grad_dtype)
+    torch.cuda.synchronize()
+    sqa.sqa_device_status()
+    rq, rk, rv = attention_backward(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(x["do"]), causal, 1 / math.sqrt(d))
+    assert_close(f64(dq), rq, "dQ")
+    assert_close(f64(dk), rk, "dK")
+    assert_close(f64(dv), rv, "dV")
+
+
+def test_training_step_config(sqa):
+    """B=4, N=8192, H_q=8, H_kv=4, d=64, causal, seed 4: dQ, and dK/dV summed
+    over each KV head's two query heads."""
+    _check_bwd(sqa, 4, 8192, 8, 4, 64, True, seed=4)
+
+
+@pytest.mark.parametrize("B,N,H_q,H_kv,d,causal", [
+    (1, 1, 2, 1, 64, True),
+    (2, 127, 4, 2, 64, True),
+    (1, 129, 8, 2, 128, False),
+    (3, 200, 4, 4, 32, True),
+    (1, 256, 16, 1, 16, False),
+    (1, 383, 8, 4, 64, False),
+    (2, 520, 2, 1, 128, True),
+    (1, 1000, 8, 8, 64, True),
+])
+def test_bwd_shape_sweep(sqa, B, N, H_q, H_kv, d, causal):
+    _check_bwd(sqa, B, N, H_q, H_kv, d, causal, seed=2000 + N)
+
+
+def test_bwd_bf16_io(sqa):
+    _check_bwd(sqa, 2, 384, 8, 4, 64, True, seed=21, o_dtype=torch.bfloat16, grad_dtype=torch.bfloat16)
