@@ -10,6 +10,7 @@
 
 #include "sqa.h"
 #include "sqa_attn_simt.cuh"
+#include "sqa_fwd_kernel.cuh"
 #include "sqa_proj_kernel.cuh"
 #include "sqa_ptx.cuh"
 
@@ -76,13 +77,65 @@ sqa_status_t check_attn_args(const void* q, const void* k, const void* v, int B,
 // ---------------------------------------------------------------------------
 // Attention forward
 // ---------------------------------------------------------------------------
+CUtensorMapSwizzle tma_swizzle_for_row_bytes(int row_bytes) {
+  return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : (row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+}
+
+// Packing factor: the largest power of two dividing G, at most 128.
+int head_pack(int G) {
+  int g = 1;
+  while (g < 128 && (G % (2 * g)) == 0) g *= 2;
+  return g;
+}
+
 template <int D>
-void launch_fwd_simt(const void* q, const void* k, const void* v, void* out, int out_bf16, float* lse, int B, int N,
-                     int H_q, int H_kv, int causal, float scale, cudaStream_t st) {
-  dim3 grid((N + sqa::kSimtRows - 1) / sqa::kSimtRows, H_q, B);
-  sqa::attn_fwd_simt_kernel<D><<<grid, sqa::kSimtRows, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-      static_cast<const __nv_bfloat16*>(v), out, out_bf16, lse, N, H_q, H_kv, causal, scale);
+sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* out, int out_bf16, float* lse, int B,
+                           int N, int H_q, int H_kv, int causal, float scale, cudaStream_t st) {
+  using C = sqa::FwdCfg<D>;
+  const int G = H_q / H_kv;
+  const int g = head_pack(G);
+  int log2g = 0;
+  while ((1 << log2g) < g) ++log2g;
+  const int T = 128 / g;
+  const CUtensorMapSwizzle swz = tma_swizzle_for_row_bytes(C::kRowBytes);
+  CUtensorMap mq, mk, mv;
+  {
+    const uint64_t dims[4] = {uint64_t(D), uint64_t(H_q), uint64_t(N), uint64_t(B)};
+    const uint64_t strides[3] = {uint64_t(D) * 2, uint64_t(H_q) * D * 2, uint64_t(N) * H_q * D * 2};
+    const uint32_t box[4] = {uint32_t(C::kRowElems), uint32_t(g), uint32_t(T), 1};
+    if (!make_map_bf16(&mq, q, 4, dims, strides, box, swz)) return SQA_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[4] = {uint64_t(D), uint64_t(H_kv), uint64_t(N), uint64_t(B)};
+    const uint64_t strides[3] = {uint64_t(D) * 2, uint64_t(H_kv) * D * 2, uint64_t(N) * H_kv * D * 2};
+    const uint32_t box[4] = {uint32_t(C::kRowElems), 1, 128, 1};
+    if (!make_map_bf16(&mk, k, 4, dims, strides, box, swz)) return SQA_ERR_CUDA;
+    if (!make_map_bf16(&mv, v, 4, dims, strides, box, swz)) return SQA_ERR_CUDA;
+  }
+  sqa::FwdParams p;
+  p.out = out;
+  p.lse = lse;
+  p.B = B;
+  p.N = N;
+  p.H_q = H_q;
+  p.H_kv = H_kv;
+  p.G = G;
+  p.g = g;
+  p.log2g = log2g;
+  p.n_sub = G / g;
+  p.n_tblk = (N + 2 * T - 1) / (2 * T);
+  p.causal = causal ? 1 : 0;
+  p.out_bf16 = out_bf16;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const long long gy = static_cast<long long>(H_kv) * p.n_sub;
+  if (gy > 65535 || B > 65535) return SQA_ERR_UNSUPPORTED;
+  auto kern = sqa::sqa_fwd_kernel<D>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+    return SQA_ERR_CUDA;
+  dim3 grid(p.n_tblk, static_cast<unsigned>(gy), B);
+  kern<<<grid, sqa::kFwdThreads, C::kSmemBytes, st>>>(mq, mk, mv, p);
+  return launch_status();
 }
 
 sqa_status_t attn_fwd_impl(const void* q, const void* k, const void* v, void* out, sqa_dtype_t out_dtype, float* lse,
@@ -94,12 +147,11 @@ sqa_status_t attn_fwd_impl(const void* q, const void* k, const void* v, void* ou
   const int ob = out_dtype == SQA_DT_BF16;
   cudaStream_t st = as_stream(stream);
   switch (d) {
-    case 16: launch_fwd_simt<16>(q, k, v, out, ob, lse, B, N, H_q, H_kv, causal, scale, st); break;
-    case 32: launch_fwd_simt<32>(q, k, v, out, ob, lse, B, N, H_q, H_kv, causal, scale, st); break;
-    case 64: launch_fwd_simt<64>(q, k, v, out, ob, lse, B, N, H_q, H_kv, causal, scale, st); break;
-    default: launch_fwd_simt<128>(q, k, v, out, ob, lse, B, N, H_q, H_kv, causal, scale, st); break;
+    case 16: return launch_fwd_tc<16>(q, k, v, out, ob, lse, B, N, H_q, H_kv, causal, scale, st);
+    case 32: return launch_fwd_tc<32>(q, k, v, out, ob, lse, B, N, H_q, H_kv, causal, scale, st);
+    case 64: return launch_fwd_tc<64>(q, k, v, out, ob, lse, B, N, H_q, H_kv, causal, scale, st);
+    default: return launch_fwd_tc<128>(q, k, v, out, ob, lse, B, N, H_q, H_kv, causal, scale, st);
   }
-  return launch_status();
 }
 
 // ---------------------------------------------------------------------------
