@@ -184,6 +184,57 @@ def run_reference(args):
 # ----------------------------------------------------------------------------
 # GPU arm
 # ----------------------------------------------------------------------------
+TRAIN = {"B": 4, "N": 8192, "H_q": 8, "H_kv": 4, "d_head": 64, "causal": True}
+
+
+def time_training_step(sqa, torch, stream, flush, dev, reps=5):
+    """Causal SQA core forward + backward at B=4, N=8192, H_q=8, H_kv=4, d=64
+    (bf16 inputs, fp32 gradients): median over reps, L2 flushed before each."""
+    from sqa_inputs import attention_inputs
+
+    t = TRAIN
+    B, N, H_q, H_kv, d = t["B"], t["N"], t["H_q"], t["H_kv"], t["d_head"]
+    scale = 1 / math.sqrt(d)
+    x = attention_inputs(B, N, H_q, H_kv, d, seed=4, with_dout=True, device=dev)
+    o = torch.empty((B, N, H_q, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H_q, N), dtype=torch.float32, device=dev)
+    dq = torch.empty((B, N, H_q, d), dtype=torch.float32, device=dev)
+    dk = torch.empty((B, N, H_kv, d), dtype=torch.float32, device=dev)
+    dv = torch.empty_like(dk)
+    wsb = sqa.sqa_attn_bwd_workspace_size(B, N, H_q, H_kv, d)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+
+    def fwd():
+        sqa.sqa_attn_fwd_ex(x["q"], x["k"], x["v"], o, sqa.SQA_DT_BF16, lse, B, N, H_q, H_kv, d, True, scale,
+                            stream=stream)
+
+    def bwd():
+        sqa.sqa_attn_bwd(x["q"], x["k"], x["v"], o, sqa.SQA_DT_BF16, x["do"], lse, dq, dk, dv, sqa.SQA_DT_F32,
+                         B, N, H_q, H_kv, d, True, scale, ws, wsb, stream=stream)
+
+    for _ in range(3):
+        fwd()
+        bwd()
+    tf, tb = [], []
+    for _ in range(reps):
+        flush.fill_(2)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        fwd()
+        e[1].record(stream)
+        bwd()
+        e[2].record(stream)
+        e[2].synchronize()
+        tf.append(e[0].elapsed_time(e[1]))
+        tb.append(e[1].elapsed_time(e[2]))
+    sqa.sqa_device_status(stream)
+    ms_f, ms_b = statistics.median(tf), statistics.median(tb)
+    f_fwd = attn_fwd_flops(B, N, H_q, d, True)
+    f_bwd = 2 * f_fwd  # dP, dV, dQ, dK; recomputation of S not credited
+    return {"config": dict(t), "fwd_ms": ms_f, "bwd_ms": ms_b, "fwd_tflops": f_fwd / ms_f / 1e9,
+            "bwd_tflops": f_bwd / ms_b / 1e9, "bwd_tflops_fa_convention": 2.5 * f_fwd / ms_b / 1e9,
+            "step_tflops": (f_fwd + f_bwd) / (ms_f + ms_b) / 1e9,
+            "tokens_per_s": B * N / ((ms_f + ms_b) / 1e3)}
 def run_sqa(args):
     import torch
     import torch.distributed as dist
@@ -296,6 +347,7 @@ def run_sqa(args):
         variants[name]["speedup_vs_mha"] = variants["MHA"]["ms"] / variants[name]["ms"]
         variants[name]["ideal_speedup"] = VARIANTS["MHA"][0] / variants[name]["H_q"]
     sqa.sqa_device_status(stream)
+    training = time_training_step(sqa, torch, stream, flush, dev)
 
     peak, peak_kind = load_peaks()
     achieved = flops_step / (statistics.mean(per_launch_ms) / 1e3) / 1e12
@@ -314,6 +366,7 @@ def run_sqa(args):
                 "steps": e2e_steps},
         "gpu_launches": args.steps,
         "variants": variants,
+        "training_step": training,
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

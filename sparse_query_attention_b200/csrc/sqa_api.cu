@@ -9,7 +9,7 @@
 #include <mutex>
 
 #include "sqa.h"
-#include "sqa_attn_simt.cuh"
+#include "sqa_bwd_kernel.cuh"
 #include "sqa_fwd_kernel.cuh"
 #include "sqa_proj_kernel.cuh"
 #include "sqa_ptx.cuh"
@@ -157,40 +157,119 @@ sqa_status_t attn_fwd_impl(const void* q, const void* k, const void* v, void* ou
 // ---------------------------------------------------------------------------
 // Attention backward
 // ---------------------------------------------------------------------------
-size_t bwd_workspace_bytes(int B, int N, int H_q) {
-  const size_t rows = static_cast<size_t>(B) * H_q * N;
+// Workspace: D and LSE*log2(e), each [B, H_q, n_pad] fp32, n_pad = N rounded
+// up to 128 so every tile the kernels touch is in bounds.
+int bwd_n_pad(int N) { return (N + 127) / 128 * 128; }
+
+size_t bwd_half_bytes(int B, int N, int H_q) {
+  const size_t rows = static_cast<size_t>(B) * H_q * bwd_n_pad(N);
   return ((rows * sizeof(float)) + 255) & ~size_t(255);
 }
 
+size_t bwd_workspace_bytes(int B, int N, int H_q) { return 2 * bwd_half_bytes(B, N, H_q); }
+
+bool make_map_f32_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner) {
+  if (!encode_fn_ready()) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * 4};
+  const cuuint32_t box[2] = {box_inner, 1};
+  const cuuint32_t es[2] = {1, 1};
+  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 [B, N, H, D] viewed as the 4-D map {D, H, N, B}, box {row, heads, tokens, 1}.
+template <int D>
+bool make_map_bnhd(CUtensorMap* map, const void* base, int B, int N, int H, uint32_t box_heads,
+                   uint32_t box_tokens) {
+  constexpr int kRowElems = D < 64 ? D : 64;
+  const uint64_t dims[4] = {uint64_t(D), uint64_t(H), uint64_t(N), uint64_t(B)};
+  const uint64_t strides[3] = {uint64_t(D) * 2, uint64_t(H) * D * 2, uint64_t(N) * H * D * 2};
+  const uint32_t box[4] = {uint32_t(kRowElems), box_heads, box_tokens, 1};
+  return make_map_bf16(map, base, 4, dims, strides, box, tma_swizzle_for_row_bytes(kRowElems * 2));
+}
+
 template <int D, typename GradT>
-void launch_bwd_simt(const void* q, const void* k, const void* v, const void* o, int o_bf16, const void* dout,
-                     const float* lse, void* dq, void* dk, void* dv, int B, int N, int H_q, int H_kv, int causal,
-                     float scale, float* dsum, cudaStream_t st) {
-  const auto* qb = static_cast<const __nv_bfloat16*>(q);
-  const auto* kb = static_cast<const __nv_bfloat16*>(k);
-  const auto* vb = static_cast<const __nv_bfloat16*>(v);
-  const auto* gb = static_cast<const __nv_bfloat16*>(dout);
-  const size_t rows = static_cast<size_t>(B) * N * H_q;
-  const unsigned dot_blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
-  sqa::attn_bwd_dot_kernel<D><<<dot_blocks, 256, 0, st>>>(o, o_bf16, gb, dsum, B, N, H_q);
-  dim3 gq((N + sqa::kSimtRows - 1) / sqa::kSimtRows, H_q, B);
-  sqa::attn_bwd_dq_simt_kernel<D, GradT><<<gq, sqa::kSimtRows, 0, st>>>(qb, kb, vb, gb, lse, dsum,
-                                                                          static_cast<GradT*>(dq), N, H_q, H_kv,
-                                                                          causal, scale);
-  dim3 gk((N + sqa::kSimtRows - 1) / sqa::kSimtRows, H_kv, B);
-  sqa::attn_bwd_dkdv_simt_kernel<D, GradT><<<gk, sqa::kSimtRows, 0, st>>>(
-      qb, kb, vb, gb, lse, dsum, static_cast<GradT*>(dk), static_cast<GradT*>(dv), N, H_q, H_kv, causal, scale);
+sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const void* o, int o_bf16, const void* dout,
+                           const float* lse, void* dq, void* dk, void* dv, int B, int N, int H_q, int H_kv,
+                           int causal, float scale, void* workspace, cudaStream_t st) {
+  const int n_pad = bwd_n_pad(N);
+  float* dsum = static_cast<float*>(workspace);
+  float* lse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + bwd_half_bytes(B, N, H_q));
+  const int G = H_q / H_kv;
+  const int g = head_pack(G);
+  int log2g = 0;
+  while ((1 << log2g) < g) ++log2g;
+  const int T = 128 / g;
+
+  sqa::BwdParams p;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.dsum = dsum;
+  p.lse2 = lse2;
+  p.B = B;
+  p.N = N;
+  p.H_q = H_q;
+  p.H_kv = H_kv;
+  p.G = G;
+  p.n_pad = n_pad;
+  p.g = g;
+  p.log2g = log2g;
+  p.n_sub = G / g;
+  p.n_tblk = (N + T - 1) / T;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const long long gy = static_cast<long long>(H_kv) * p.n_sub;
+  if (gy > 65535 || B > 65535) return SQA_ERR_UNSUPPORTED;
+
+  CUtensorMap m_k128, m_v128, m_q64, m_do64, m_l2, m_ds, m_qp, m_dop, m_k64, m_v64;
+  if (!make_map_bnhd<D>(&m_k128, k, B, N, H_kv, 1, 128) || !make_map_bnhd<D>(&m_v128, v, B, N, H_kv, 1, 128) ||
+      !make_map_bnhd<D>(&m_q64, q, B, N, H_q, 1, 64) || !make_map_bnhd<D>(&m_do64, dout, B, N, H_q, 1, 64) ||
+      !make_map_bnhd<D>(&m_qp, q, B, N, H_q, g, T) || !make_map_bnhd<D>(&m_dop, dout, B, N, H_q, g, T) ||
+      !make_map_bnhd<D>(&m_k64, k, B, N, H_kv, 1, 64) || !make_map_bnhd<D>(&m_v64, v, B, N, H_kv, 1, 64) ||
+      !make_map_f32_2d(&m_l2, lse2, n_pad, uint64_t(B) * H_q, 64) ||
+      !make_map_f32_2d(&m_ds, dsum, n_pad, uint64_t(B) * H_q, 64))
+    return SQA_ERR_CUDA;
+
+  // 1. D and LSE in log2 units.
+  const size_t prep_rows = static_cast<size_t>(B) * H_q * n_pad;
+  sqa::bwd_prep_kernel<D><<<static_cast<unsigned>((prep_rows * 32 + 255) / 256), 256, 0, st>>>(
+      o, o_bf16, static_cast<const __nv_bfloat16*>(dout), lse, dsum, lse2, B, N, H_q, n_pad);
+  if (cudaGetLastError() != cudaSuccess) return SQA_ERR_CUDA;
+
+  // 2. dK, dV (KV-outer).
+  {
+    auto kern = sqa::bwd_dkdv_kernel<D, GradT>;
+    constexpr int smem = sqa::DkdvCfg<D>::kSmemBytes;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return SQA_ERR_CUDA;
+    dim3 grid((N + 127) / 128, H_kv, B);
+    kern<<<grid, sqa::kBwdThreads, smem, st>>>(m_k128, m_v128, m_q64, m_do64, m_l2, m_ds, p);
+    if (cudaGetLastError() != cudaSuccess) return SQA_ERR_CUDA;
+  }
+  // 3. dQ (Q-outer).
+  {
+    auto kern = sqa::bwd_dq_kernel<D, GradT>;
+    constexpr int smem = sqa::DqCfg<D>::kSmemBytes;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return SQA_ERR_CUDA;
+    dim3 grid(p.n_tblk, static_cast<unsigned>(gy), B);
+    kern<<<grid, sqa::kBwdThreads, smem, st>>>(m_qp, m_dop, m_k64, m_v64, p);
+  }
+  return launch_status();
 }
 
 template <int D>
-void launch_bwd_d(bool grad_bf16, const void* q, const void* k, const void* v, const void* o, int o_bf16,
-                  const void* dout, const float* lse, void* dq, void* dk, void* dv, int B, int N, int H_q, int H_kv,
-                  int causal, float scale, float* dsum, cudaStream_t st) {
+sqa_status_t launch_bwd_d(bool grad_bf16, const void* q, const void* k, const void* v, const void* o, int o_bf16,
+                          const void* dout, const float* lse, void* dq, void* dk, void* dv, int B, int N, int H_q,
+                          int H_kv, int causal, float scale, void* ws, cudaStream_t st) {
   if (grad_bf16)
-    launch_bwd_simt<D, __nv_bfloat16>(q, k, v, o, o_bf16, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale,
-                                      dsum, st);
-  else
-    launch_bwd_simt<D, float>(q, k, v, o, o_bf16, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, dsum, st);
+    return launch_bwd_tc<D, __nv_bfloat16>(q, k, v, o, o_bf16, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal,
+                                           scale, ws, st);
+  return launch_bwd_tc<D, float>(q, k, v, o, o_bf16, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, ws, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -261,17 +340,15 @@ sqa_status_t sqa_attn_bwd(const void* q, const void* k, const void* v, const voi
   if ((o_dtype != SQA_DT_F32 && o_dtype != SQA_DT_BF16) || (grad_dtype != SQA_DT_F32 && grad_dtype != SQA_DT_BF16))
     return SQA_ERR_INVALID_ARG;
   if (workspace_bytes < bwd_workspace_bytes(B, N, H_q)) return SQA_ERR_INVALID_ARG;
-  float* dsum = static_cast<float*>(workspace);
   const bool gb = grad_dtype == SQA_DT_BF16;
   const int ob = o_dtype == SQA_DT_BF16;
   cudaStream_t st = as_stream(stream);
   switch (d_head) {
-    case 16: launch_bwd_d<16>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, dsum, st); break;
-    case 32: launch_bwd_d<32>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, dsum, st); break;
-    case 64: launch_bwd_d<64>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, dsum, st); break;
-    default: launch_bwd_d<128>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, dsum, st); break;
+    case 16: return launch_bwd_d<16>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, workspace, st);
+    case 32: return launch_bwd_d<32>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, workspace, st);
+    case 64: return launch_bwd_d<64>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, workspace, st);
+    default: return launch_bwd_d<128>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, workspace, st);
   }
-  return launch_status();
 }
 
 sqa_status_t sqa_proj(const void* x, const void* w, const float* bias, void* y, sqa_dtype_t y_dtype, int M, int K,

@@ -1,0 +1,572 @@
+// sqa_bwd_kernel.cuh - gradient of the Sparse Query Attention core on sm_100a.
+//
+// With P_tu = exp(s_tu - LSE_t), s_tu = scale <q_t, k_u>, D_t = <dO_t, O_t>:
+//   dV_j = sum_{h in group j} P^T dO_h
+//   dS   = P o (dO_h V_j^T - D)
+//   dQ_h = scale dS K_j
+//   dK_j = scale sum_{h in group j} dS^T Q_h
+// The training-time gains the pages report ("ReactiveAI/GQA-Ref-Micro" model
+// card, results; "Sparse Query Attention (SQA): ...", abstract: pre-training
+// and fine-tuning) come from these contractions also running over H_q heads
+// only.
+//
+// Three kernels, all launched on one stream, no atomics (deterministic):
+//   bwd_prep_kernel   D_t and LSE_t * log2(e) into a padded fp32 workspace.
+//   bwd_dkdv_kernel   KV-outer: one CTA per 128-key tile of one KV head; the
+//                     keys are the TMEM lanes and the loop runs over every
+//                     query head of the group and every 64-token query
+//                     sub-tile, so the group sum of dK/dV happens inside one
+//                     TMEM accumulator.  Per step: S^T = K Q^T and
+//                     dP^T = V dO^T (tcgen05, SMEM x SMEM), softmax warps form
+//                     P^T and dS^T in bf16 back in TMEM, then dV += P^T dO and
+//                     dK += dS^T Q (A operand from TMEM).
+//   bwd_dq_kernel     Q-outer: one CTA per 128 packed query rows (as in the
+//                     forward); per 64-key sub-tile: S = Q K^T, dP = dO V^T,
+//                     dS in TMEM, dQ += dS K.
+// Score tiles are 64 wide and double-buffered in TMEM so that the softmax of
+// one buffer overlaps the tensor-core work on the other.
+#pragma once
+
+#include "sqa_ptx.cuh"
+
+namespace sqa {
+
+// ---------------------------------------------------------------------------
+// Preprocess: D[b,h,t] = sum_c dO[b,t,h,c] O[b,t,h,c]; L2[b,h,t] = LSE * log2 e.
+// Workspace rows are padded to n_pad tokens (multiple of 128) with zeros.
+// One warp per (b, h, t) of the padded space.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void bwd_prep_kernel(const void* __restrict__ o, int o_bf16, const __nv_bfloat16* __restrict__ dout,
+                                const float* __restrict__ lse, float* __restrict__ dsum, float* __restrict__ lse2,
+                                int B, int N, int H_q, int n_pad) {
+  const size_t idx = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+  const int lane = threadIdx.x & 31;
+  const size_t total = static_cast<size_t>(B) * H_q * n_pad;
+  if (idx >= total) return;
+  const int t = static_cast<int>(idx % n_pad);
+  const size_t bh = idx / n_pad;
+  const int h = static_cast<int>(bh % H_q);
+  const int b = static_cast<int>(bh / H_q);
+  float acc = 0.f, l2 = 0.f;
+  if (t < N) {
+    const size_t row = ((static_cast<size_t>(b) * N + t) * H_q + h) * D;
+    for (int c = lane; c < D; c += 32) {
+      const float ov = o_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(o)[row + c])
+                              : static_cast<const float*>(o)[row + c];
+      acc = fmaf(ov, __bfloat162float(dout[row + c]), acc);
+    }
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+    l2 = lse[bh * N + t] * 1.4426950408889634f;
+  }
+  if (lane == 0) {
+    dsum[idx] = acc;
+    lse2[idx] = l2;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void store16(T* dst, const float (&v)[16]);
+template <>
+__device__ __forceinline__ void store16<float>(float* dst, const float (&v)[16]) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+template <>
+__device__ __forceinline__ void store16<__nv_bfloat16>(__nv_bfloat16* dst, const float (&v)[16]) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+  d4[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                     pack_bf16x2(v[6], v[7]));
+  d4[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
+                     pack_bf16x2(v[14], v[15]));
+}
+
+// Swizzled-tile geometry shared by the backward kernels: R rows of D bf16,
+// stored as D/64 column chunks of R rows x (up to) 128 bytes.
+template <int D, int R>
+struct TileGeo {
+  static constexpr int kRowElems = D < 64 ? D : 64;
+  static constexpr int kRowBytes = kRowElems * 2;
+  static constexpr int kChunks = D / kRowElems;
+  static constexpr int kChunkBytes = R * kRowBytes;
+  static constexpr int kBytes = kChunks * kChunkBytes;
+  static constexpr uint32_t kSwizzle = kRowBytes == 128 ? kSw128 : (kRowBytes == 64 ? kSw64 : kSw32);
+  static constexpr uint32_t kSbo = 8 * kRowBytes;
+
+  // K-major operand (rows = M or N, K = D): descriptor for the 16-wide K step kk.
+  __device__ static uint64_t kmajor(uint32_t base, int kk) {
+    const int c = (kk * 16) / kRowElems;
+    const uint32_t off = c * kChunkBytes + ((kk * 16) % kRowElems) * 2;
+    return smem_desc(base + off, 16, kSbo, kSwizzle);
+  }
+  // MN-major operand (N = D along the row, K = rows): descriptor for rows
+  // [16 kk, 16 kk + 16).
+  __device__ static uint64_t mnmajor(uint32_t base, int kk) {
+    return smem_desc(base + kk * 16 * kRowBytes, kChunkBytes, kSbo, kSwizzle);
+  }
+};
+
+struct BwdParams {
+  void* dq;
+  void* dk;
+  void* dv;
+  const float* dsum;  // [B, H_q, n_pad]
+  const float* lse2;  // [B, H_q, n_pad]
+  int B, N, H_q, H_kv, G, n_pad;
+  int g, log2g, n_sub, n_tblk;  // packing of the dQ kernel
+  int causal;
+  float scale;
+  float scale_log2;
+};
+
+constexpr int kBwdThreads = 384;
+
+// ===========================================================================
+// dK / dV
+// ===========================================================================
+template <int D>
+struct DkdvCfg {
+  using KV = TileGeo<D, 128>;  // resident K and V tiles
+  using QT = TileGeo<D, 64>;   // streamed Q / dO sub-tiles
+  static constexpr int kStages = 4;
+  static constexpr int kStatBytes = 1024;                        // LSE2 (256 B) + D (256 B), 1 KB aligned
+  static constexpr int kStageBytes = 2 * QT::kBytes + kStatBytes;  // Q, dO, stats
+  static constexpr int kSmemBytes = 2 * KV::kBytes + kStages * kStageBytes + 1024;
+  // TMEM columns: S^T/P^T and dP^T/dS^T of buffer b, then dV and dK.
+  __device__ static constexpr uint32_t col_s(int b) { return 128u * b; }
+  __device__ static constexpr uint32_t col_dp(int b) { return 64u + 128u * b; }
+  static constexpr uint32_t kColDV = 256, kColDK = 256 + D;
+};
+
+template <int D, typename GradT>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ CUtensorMap tm_lse2, const __grid_constant__ CUtensorMap tm_dsum,
+                    const BwdParams p) {
+  using C = DkdvCfg<D>;
+  using KV = typename C::KV;
+  using QT = typename C::QT;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t kv_full;
+  __shared__ __align__(8) uint64_t st_full[C::kStages];
+  __shared__ __align__(8) uint64_t st_empty[C::kStages];
+  __shared__ __align__(8) uint64_t s_full[2];
+  __shared__ __align__(8) uint64_t p_ready[2];
+  __shared__ __align__(8) uint64_t mma_done;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* k_smem = smem;
+  uint8_t* v_smem = smem + KV::kBytes;
+  uint8_t* stages = smem + 2 * KV::kBytes;
+
+  const int warp = warp_id_uniform();
+  const int lane = threadIdx.x & 31;
+  const int kt = blockIdx.x;  // key tile
+  const int j = blockIdx.y;
+  const int b = blockIdx.z;
+  const int key0 = kt * 128;
+  const int n_qsub = (p.N + 63) / 64;
+  const int qs_begin = p.causal ? (key0 / 64) : 0;
+  const int per_head = n_qsub - qs_begin;
+  const int n_steps = p.G * per_head;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&kv_full, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&st_full[s], 1);
+      mbar_init(&st_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_ready[t], 4);
+    }
+    mbar_init(&mma_done, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(&tmem_base_sh, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      mbar_arrive_expect_tx(&kv_full, 2 * KV::kBytes);
+      for (int c = 0; c < KV::kChunks; ++c) {
+        tma_load_4d(&tm_k, &kv_full, k_smem + c * KV::kChunkBytes, c * KV::kRowElems, j, key0, b);
+        tma_load_4d(&tm_v, &kv_full, v_smem + c * KV::kChunkBytes, c * KV::kRowElems, j, key0, b);
+      }
+      int s = 0;
+      for (; s < n_steps; ++s) {
+        const int st = s % C::kStages;
+        if (s >= C::kStages && !mbar_wait(&st_empty[st], ((s / C::kStages) - 1) & 1, &abort_flag)) break;
+        const int h = j * p.G + s / per_head;
+        const int q0 = (qs_begin + s % per_head) * 64;
+        uint8_t* dst = stages + st * C::kStageBytes;
+        mbar_arrive_expect_tx(&st_full[st], 2 * QT::kBytes + 512);
+        for (int c = 0; c < QT::kChunks; ++c) {
+          tma_load_4d(&tm_q, &st_full[st], dst + c * QT::kChunkBytes, c * QT::kRowElems, h, q0, b);
+          tma_load_4d(&tm_do, &st_full[st], dst + QT::kBytes + c * QT::kChunkBytes, c * QT::kRowElems, h, q0, b);
+        }
+        const int stat_row = b * p.H_q + h;
+        tma_load_2d(&tm_lse2, &st_full[st], dst + 2 * QT::kBytes, q0, stat_row);
+        tma_load_2d(&tm_dsum, &st_full[st], dst + 2 * QT::kBytes + 256, q0, stat_row);
+      }
+      mbar_drain(&kv_full, 0);
+      for (int l = max(0, s - C::kStages); l < s; ++l) mbar_drain(&st_full[l % C::kStages], (l / C::kStages) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);  // M=128 keys, N=64 queries
+      constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, 0, 1);   // M=128 keys, N=D, B MN-major
+      const uint32_t k_addr = smem_addr(k_smem), v_addr = smem_addr(v_smem);
+      const uint32_t st_addr = smem_addr(stages);
+      auto issue_scores = [&](int s) {
+        const int buf = s & 1;
+        const uint32_t qa = st_addr + (s % C::kStages) * C::kStageBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + C::col_s(buf), KV::kmajor(k_addr, kk), QT::kmajor(qa, kk), idesc_s, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + C::col_dp(buf), KV::kmajor(v_addr, kk), QT::kmajor(qa + QT::kBytes, kk), idesc_s, kk > 0);
+        mma_commit(&s_full[buf]);
+      };
+      bool ok = mbar_wait(&kv_full, 0, &abort_flag);
+      for (int s = 0; s < 2 && s < n_steps && ok; ++s) {
+        ok = mbar_wait(&st_full[s % C::kStages], (s / C::kStages) & 1, &abort_flag);
+        if (ok) {
+          tc_fence_after();
+          issue_scores(s);
+        }
+      }
+      for (int s = 0; s < n_steps && ok; ++s) {
+        const int buf = s & 1;
+        if (!mbar_wait(&p_ready[buf], (s >> 1) & 1, &abort_flag)) break;
+        tc_fence_after();
+        const uint32_t qa = st_addr + (s % C::kStages) * C::kStageBytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // 64 query rows = 4 x K16
+          mma_ts(tmem + C::kColDV, tmem + C::col_s(buf) + kk * 8, QT::mnmajor(qa + QT::kBytes, kk), idesc_g,
+                 (s > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tmem + C::kColDK, tmem + C::col_dp(buf) + kk * 8, QT::mnmajor(qa, kk), idesc_g,
+                 (s > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&st_empty[s % C::kStages]);
+        if (s + 2 < n_steps) {
+          if (!mbar_wait(&st_full[(s + 2) % C::kStages], ((s + 2) / C::kStages) & 1, &abort_flag)) break;
+          tc_fence_after();
+          issue_scores(s + 2);
+        }
+      }
+      mma_commit(&mma_done);
+    }
+  } else if (warp >= 4) {
+    // ---------------- softmax-gradient warps ----------------
+    const int grp = (warp - 4) >> 2;  // handles steps s with s % 2 == grp
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;  // key row
+    const int u = key0 + r;        // key token
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int s = grp; s < n_steps; s += 2) {
+      if (!mbar_wait(&s_full[grp], (s >> 1) & 1, &abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[64], dr[64];
+      tmem_ld32(lane_base + C::col_s(grp), *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(lane_base + C::col_s(grp) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(lane_base + C::col_dp(grp), *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+      tmem_ld32(lane_base + C::col_dp(grp) + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+      const uint8_t* stat = stages + (s % C::kStages) * C::kStageBytes + 2 * QT::kBytes;
+      const float* l2 = reinterpret_cast<const float*>(stat);
+      const float* dd = reinterpret_cast<const float*>(stat + 256);
+      const int q0 = (qs_begin + s % per_head) * 64;
+      // Query column c (token q0 + c) contributes iff q0 + c < N and, when
+      // causal, q0 + c >= u.
+      int lo = p.causal ? u - q0 : 0;          // first allowed column
+      const int hi = p.N - q0;                 // columns [0, hi) are < N
+      tmem_wait_ld();
+      uint32_t pk[32], dk[32];
+#pragma unroll
+      for (int c2 = 0; c2 < 32; ++c2) {
+        float pv[2], dsv[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = 2 * c2 + e;
+          const bool keep = c >= lo && c < hi;
+          const float pr = ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, -l2[c]));
+          pv[e] = keep ? pr : 0.f;
+          dsv[e] = keep ? pr * (__uint_as_float(dr[c]) - dd[c]) : 0.f;
+        }
+        pk[c2] = pack_bf16x2(pv[0], pv[1]);
+        dk[c2] = pack_bf16x2(dsv[0], dsv[1]);
+      }
+      tmem_st32(lane_base + C::col_s(grp), pk);
+      tmem_st32(lane_base + C::col_dp(grp), dk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_ready[grp]);
+    }
+    // ---------------- epilogue: group 0 writes dV, group 1 writes dK --------
+    if (ok) ok = mbar_wait(&mma_done, 0, &abort_flag);
+    if (ok) {
+      tc_fence_after();
+      const bool valid = u < p.N;
+      const uint32_t col = grp == 0 ? C::kColDV : C::kColDK;
+      const float mult = grp == 0 ? 1.f : p.scale;
+      GradT* dst = static_cast<GradT*>(grp == 0 ? p.dv : p.dk) +
+                   ((static_cast<size_t>(b) * p.N + (valid ? u : 0)) * p.H_kv + j) * D;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 16) {
+        uint32_t rr[16];
+        tmem_ld16(lane_base + col + c0, rr);
+        tmem_wait_ld();
+        float v[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) v[c] = (n_steps > 0 ? __uint_as_float(rr[c]) : 0.f) * mult;
+        if (valid) store16<GradT>(dst + c0, v);
+      }
+    }
+  }
+
+  __syncwarp();
+  if (threadIdx.x == 32) mbar_drain(&mma_done, 0);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ===========================================================================
+// dQ
+// ===========================================================================
+template <int D>
+struct DqCfg {
+  using QT = TileGeo<D, 128>;  // resident Q and dO tiles (packed rows)
+  using KS = TileGeo<D, 64>;   // streamed K / V sub-tiles
+  static constexpr int kStages = 4;
+  static constexpr int kStageBytes = 2 * KS::kBytes;
+  static constexpr int kSmemBytes = 2 * QT::kBytes + kStages * kStageBytes + 1024;
+  // TMEM columns: S/dS and dP of buffer b, then dQ.
+  __device__ static constexpr uint32_t col_s(int b) { return 128u * b; }
+  __device__ static constexpr uint32_t col_dp(int b) { return 64u + 128u * b; }
+  static constexpr uint32_t kColDQ = 256;
+};
+
+template <int D, typename GradT>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const BwdParams p) {
+  using C = DqCfg<D>;
+  using QT = typename C::QT;
+  using KS = typename C::KS;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t q_full;
+  __shared__ __align__(8) uint64_t st_full[C::kStages];
+  __shared__ __align__(8) uint64_t st_empty[C::kStages];
+  __shared__ __align__(8) uint64_t s_full[2];
+  __shared__ __align__(8) uint64_t p_ready[2];
+  __shared__ __align__(8) uint64_t mma_done;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_smem = smem;
+  uint8_t* do_smem = smem + QT::kBytes;
+  uint8_t* stages = smem + 2 * QT::kBytes;
+
+  const int warp = warp_id_uniform();
+  const int lane = threadIdx.x & 31;
+  const int T = 128 >> p.log2g;
+  const int tblk = p.causal ? (p.n_tblk - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
+  const int j = blockIdx.y / p.n_sub;
+  const int sub = blockIdx.y % p.n_sub;
+  const int b = blockIdx.z;
+  const int h0 = j * p.G + sub * p.g;
+  const int t0 = tblk * T;
+  const int last_tok = min(t0 + T, p.N) - 1;
+  const int n_steps = p.causal ? (last_tok / 64 + 1) : (p.N + 63) / 64;  // 64-key sub-tiles
+
+  if (threadIdx.x == 0) {
+    mbar_init(&q_full, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&st_full[s], 1);
+      mbar_init(&st_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_ready[t], 4);
+    }
+    mbar_init(&mma_done, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(&tmem_base_sh, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&q_full, 2 * QT::kBytes);
+      for (int c = 0; c < QT::kChunks; ++c) {
+        tma_load_4d(&tm_q, &q_full, q_smem + c * QT::kChunkBytes, c * QT::kRowElems, h0, t0, b);
+        tma_load_4d(&tm_do, &q_full, do_smem + c * QT::kChunkBytes, c * QT::kRowElems, h0, t0, b);
+      }
+      int s = 0;
+      for (; s < n_steps; ++s) {
+        const int st = s % C::kStages;
+        if (s >= C::kStages && !mbar_wait(&st_empty[st], ((s / C::kStages) - 1) & 1, &abort_flag)) break;
+        uint8_t* dst = stages + st * C::kStageBytes;
+        mbar_arrive_expect_tx(&st_full[st], 2 * KS::kBytes);
+        for (int c = 0; c < KS::kChunks; ++c) {
+          tma_load_4d(&tm_k, &st_full[st], dst + c * KS::kChunkBytes, c * KS::kRowElems, j, s * 64, b);
+          tma_load_4d(&tm_v, &st_full[st], dst + KS::kBytes + c * KS::kChunkBytes, c * KS::kRowElems, j, s * 64, b);
+        }
+      }
+      mbar_drain(&q_full, 0);
+      for (int l = max(0, s - C::kStages); l < s; ++l) mbar_drain(&st_full[l % C::kStages], (l / C::kStages) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);  // M=128 rows, N=64 keys
+      constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, 0, 1);   // M=128 rows, N=D, B MN-major
+      const uint32_t q_addr = smem_addr(q_smem), do_addr = smem_addr(do_smem);
+      const uint32_t st_addr = smem_addr(stages);
+      auto issue_scores = [&](int s) {
+        const int buf = s & 1;
+        const uint32_t ka = st_addr + (s % C::kStages) * C::kStageBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + C::col_s(buf), QT::kmajor(q_addr, kk), KS::kmajor(ka, kk), idesc_s, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + C::col_dp(buf), QT::kmajor(do_addr, kk), KS::kmajor(ka + KS::kBytes, kk), idesc_s, kk > 0);
+        mma_commit(&s_full[buf]);
+      };
+      bool ok = mbar_wait(&q_full, 0, &abort_flag);
+      for (int s = 0; s < 2 && s < n_steps && ok; ++s) {
+        ok = mbar_wait(&st_full[s % C::kStages], (s / C::kStages) & 1, &abort_flag);
+        if (ok) {
+          tc_fence_after();
+          issue_scores(s);
+        }
+      }
+      for (int s = 0; s < n_steps && ok; ++s) {
+        const int buf = s & 1;
+        if (!mbar_wait(&p_ready[buf], (s >> 1) & 1, &abort_flag)) break;
+        tc_fence_after();
+        const uint32_t ka = st_addr + (s % C::kStages) * C::kStageBytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // 64 keys = 4 x K16
+          mma_ts(tmem + C::kColDQ, tmem + C::col_s(buf) + kk * 8, KS::mnmajor(ka, kk), idesc_g,
+                 (s > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&st_empty[s % C::kStages]);
+        if (s + 2 < n_steps) {
+          if (!mbar_wait(&st_full[(s + 2) % C::kStages], ((s + 2) / C::kStages) & 1, &abort_flag)) break;
+          tc_fence_after();
+          issue_scores(s + 2);
+        }
+      }
+      mma_commit(&mma_done);
+    }
+  } else if (warp >= 4) {
+    const int grp = (warp - 4) >> 2;
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const int tok = t0 + (r >> p.log2g);
+    const int head = h0 + (r & (p.g - 1));
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const float sl2 = p.scale_log2;
+    const size_t stat = (static_cast<size_t>(b) * p.H_q + head) * p.n_pad + tok;  // tok < n_pad
+    const float l2 = p.lse2[stat];
+    const float dd = p.dsum[stat];
+    bool ok = true;
+    for (int s = grp; s < n_steps; s += 2) {
+      if (!mbar_wait(&s_full[grp], (s >> 1) & 1, &abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[64], dr[64];
+      tmem_ld32(lane_base + C::col_s(grp), *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(lane_base + C::col_s(grp) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(lane_base + C::col_dp(grp), *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+      tmem_ld32(lane_base + C::col_dp(grp) + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+      const int kbase = s * 64;
+      int hi = p.N - kbase;                        // keys [0, hi) are < N
+      if (p.causal) hi = min(hi, tok - kbase + 1);  // keys <= tok
+      tmem_wait_ld();
+      uint32_t dk[32];
+#pragma unroll
+      for (int c2 = 0; c2 < 32; ++c2) {
+        float dsv[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = 2 * c2 + e;
+          const float pr = ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, -l2));
+          dsv[e] = c < hi ? pr * (__uint_as_float(dr[c]) - dd) : 0.f;
+        }
+        dk[c2] = pack_bf16x2(dsv[0], dsv[1]);
+      }
+      tmem_st32(lane_base + C::col_s(grp), dk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_ready[grp]);
+    }
+    if (ok) ok = mbar_wait(&mma_done, 0, &abort_flag);
+    if (ok) {
+      tc_fence_after();
+      const bool valid = tok < p.N;
+      GradT* dst = static_cast<GradT*>(p.dq) + ((static_cast<size_t>(b) * p.N + (valid ? tok : 0)) * p.H_q + head) * D;
+      // The two groups split the columns of dQ (group 0 alone when D = 16).
+      constexpr int kHalf = D >= 32 ? D / 2 : D;
+#pragma unroll 1
+      for (int c0 = grp * kHalf; c0 < (grp + 1) * kHalf && c0 < D; c0 += 16) {
+        uint32_t rr[16];
+        tmem_ld16(lane_base + C::kColDQ + c0, rr);
+        tmem_wait_ld();
+        float v[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) v[c] = (n_steps > 0 ? __uint_as_float(rr[c]) : 0.f) * p.scale;
+        if (valid) store16<GradT>(dst + c0, v);
+      }
+    }
+  }
+
+  __syncwarp();
+  if (threadIdx.x == 32) mbar_drain(&mma_done, 0);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace sqa
