@@ -379,6 +379,31 @@ def run_sqa(args):
     return 0
 
 
+def run_profile(args):
+    """Launches only the kernels of one workload, steps times, for profilers."""
+    import torch
+
+    import sparse_query_attention_b200 as sqa
+    from sqa_inputs import attention_inputs
+
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    if args.profile == "fwd":
+        w = WORKLOAD
+        B, N, H_q, H_kv, d = w["B"], w["N"], w["H_q"], w["H_kv"], w["d_head"]
+        x = attention_inputs(B, N, H_q, H_kv, d, seed=2, device=dev)
+        out = torch.empty((B, N, H_q * d), dtype=torch.float32, device=dev)
+        for _ in range(args.steps):
+            sqa.sqa_attn_fwd(x["q"], x["k"], x["v"], out, B, N, H_q, H_kv, d, w["causal"], 1 / math.sqrt(d),
+                             stream=stream)
+    else:
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        time_training_step(sqa, torch, stream, flush, dev, reps=max(1, args.steps - 3))
+    torch.cuda.synchronize(dev)
+    sqa.sqa_device_status(stream)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -386,7 +411,12 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["sqa", "reference"], default="sqa")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["fwd", "bwd"], default=None,
+                    help="only launch the kernels (for ncu): fwd = the bench workload's forward, "
+                         "bwd = the B=4, N=8192 causal training step; no timing, no JSON")
     args = ap.parse_args(argv)
+    if args.profile:
+        return run_profile(args)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args)
