@@ -106,6 +106,38 @@ sqa_status_t sqa_attn_bwd(const void* q, const void* k, const void* v,
                           void* stream);
 
 /*
+ * sqa_attn_bwd_static - sqa_attn_bwd without a caller-supplied workspace.
+ * (Library plumbing; the paper has no counterpart.)
+ *
+ * For callers that cannot allocate device memory themselves: code handed
+ * only input and output pointers by a host framework that owns the GPU's
+ * memory (a plugin or custom-op interface), or services that forbid any
+ * allocation once they are running.  The scratch the backward needs (the
+ * per-row D and LSE*log2(e) values) lives instead in one fixed device array
+ * inside this library, SQA_BWD_STATIC_SCRATCH_BYTES in size, which every GPU
+ * that loads the library holds until the process exits.
+ *
+ * Arguments, layouts and results are those of sqa_attn_bwd.  The call
+ * allocates nothing (no cudaMalloc/cudaFree, no allocating library routine).
+ * Shapes whose workspace (sqa_attn_bwd_workspace_size) exceeds
+ * SQA_BWD_STATIC_SCRATCH_BYTES return SQA_ERR_UNSUPPORTED and launch nothing.
+ * The first call on a device looks up the array's device address (with that
+ * device current); make that first call before any stream capture.  All
+ * calls share the one array: calls that overlap on the GPU (different
+ * streams, or different host threads, on the same device) race on it, so
+ * serialise them.  The array keeps the previous call's contents; the
+ * backward overwrites every entry it reads, so nothing needs clearing.
+ */
+#define SQA_BWD_STATIC_SCRATCH_BYTES (16u << 20)
+
+sqa_status_t sqa_attn_bwd_static(const void* q, const void* k, const void* v,
+                                 const void* out, sqa_dtype_t o_dtype,
+                                 const void* dout, const float* lse,
+                                 void* dq, void* dk, void* dv, sqa_dtype_t grad_dtype,
+                                 int B, int N, int H_q, int H_kv, int d_head, int causal,
+                                 float scale, void* stream);
+
+/*
  * sqa_proj - one reduced-width projection, Y[M, Nout] = X[M, K] W[Nout, K]^T
  * (+ bias), the Q/K/V projections (Nout = H_q*d_head or H_kv*d_head) and the
  * output projection (K = H_q*d_head).  X and W are bf16 (W in nn.Linear

@@ -7,7 +7,7 @@ status raises :class:`SQAError`.  Every step of the computation runs in the
 library's CUDA kernels; there is no other implementation behind these names.
 
 The library must have been built (``python -m sparse_query_attention_b200.build``);
-importing this package without it raises ImportError.
+the first call into it raises ImportError when it is missing.
 """
 
 from __future__ import annotations
@@ -34,6 +34,8 @@ SIGNATURES = {
     "sqa_attn_bwd_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "sqa_attn_bwd": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I,
                           _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
+    "sqa_attn_bwd_static": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I,
+                                 _I, _I, _I, _I, _I, _I, _F, _P]),
     "sqa_proj": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "sqa_device_status": (_I, [_P]),
     "sqa_status_string": (ctypes.c_char_p, [_I]),
@@ -59,11 +61,16 @@ def _load() -> ctypes.CDLL:
     return lib
 
 
-_lib = _load()
+_handle = None
 
 
 def library() -> ctypes.CDLL:
-    return _lib
+    """The loaded libsqa.so (loaded on first use; raises ImportError if it
+    has not been built)."""
+    global _handle
+    if _handle is None:
+        _handle = _load()
+    return _handle
 
 
 def _ptr(x):
@@ -94,11 +101,11 @@ def _check(status: int, where: str) -> None:
 
 
 def status_string(status: int) -> str:
-    return _lib.sqa_status_string(int(status)).decode()
+    return library().sqa_status_string(int(status)).decode()
 
 
 def sqa_version() -> str:
-    return _lib.sqa_version().decode()
+    return library().sqa_version().decode()
 
 
 def sqa_status_string(status: int) -> str:
@@ -106,34 +113,45 @@ def sqa_status_string(status: int) -> str:
 
 
 def sqa_attn_fwd(q, k, v, out, B, N, H_q, H_kv, d_head, causal, scale, stream=None) -> None:
-    _check(_lib.sqa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, N, H_q, H_kv, d_head,
+    _check(library().sqa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, N, H_q, H_kv, d_head,
                              int(bool(causal)), float(scale), _stream(stream)), "sqa_attn_fwd")
 
 
 def sqa_attn_fwd_ex(q, k, v, out, out_dtype, lse, B, N, H_q, H_kv, d_head, causal, scale,
                     stream=None) -> None:
-    _check(_lib.sqa_attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(out_dtype), _ptr(lse),
+    _check(library().sqa_attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(out_dtype), _ptr(lse),
                                 B, N, H_q, H_kv, d_head, int(bool(causal)), float(scale),
                                 _stream(stream)), "sqa_attn_fwd_ex")
 
 
 def sqa_attn_bwd_workspace_size(B, N, H_q, H_kv, d_head) -> int:
-    return int(_lib.sqa_attn_bwd_workspace_size(B, N, H_q, H_kv, d_head))
+    return int(library().sqa_attn_bwd_workspace_size(B, N, H_q, H_kv, d_head))
 
 
 def sqa_attn_bwd(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B, N, H_q, H_kv,
                  d_head, causal, scale, workspace, workspace_bytes, stream=None) -> None:
-    _check(_lib.sqa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(o_dtype), _ptr(dout),
+    _check(library().sqa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(o_dtype), _ptr(dout),
                              _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), int(grad_dtype),
                              B, N, H_q, H_kv, d_head, int(bool(causal)), float(scale),
                              _ptr(workspace), int(workspace_bytes), _stream(stream)),
            "sqa_attn_bwd")
 
 
+def sqa_attn_bwd_static(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B, N, H_q, H_kv,
+                        d_head, causal, scale, stream=None) -> None:
+    """sqa_attn_bwd with the library's fixed device scratch instead of a
+    caller workspace, for callers that cannot allocate device memory; see
+    include/sqa.h for its size limit and sharing rules."""
+    _check(library().sqa_attn_bwd_static(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(o_dtype), _ptr(dout),
+                                    _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), int(grad_dtype),
+                                    B, N, H_q, H_kv, d_head, int(bool(causal)), float(scale),
+                                    _stream(stream)), "sqa_attn_bwd_static")
+
+
 def sqa_proj(x, w, bias, y, y_dtype, M, K, Nout, stream=None) -> None:
-    _check(_lib.sqa_proj(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), int(y_dtype), M, K, Nout,
+    _check(library().sqa_proj(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), int(y_dtype), M, K, Nout,
                          _stream(stream)), "sqa_proj")
 
 
 def sqa_device_status(stream=None) -> None:
-    _check(_lib.sqa_device_status(_stream(stream)), "sqa_device_status")
+    _check(library().sqa_device_status(_stream(stream)), "sqa_device_status")

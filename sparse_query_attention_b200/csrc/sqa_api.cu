@@ -351,6 +351,51 @@ sqa_status_t sqa_attn_bwd(const void* q, const void* k, const void* v, const voi
   }
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Backward without a caller workspace: the scratch is this file-scope device
+// array, present on every GPU that loads the library until the process exits.
+// In host code `g_bwd_static_scratch` names a host-side shadow, never the
+// device memory: its device address comes from cudaGetSymbolAddress, looked
+// up once per device with that device current.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_bwd_static_scratch[SQA_BWD_STATIC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_static_scratch_mu;
+void* g_static_scratch_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, or null.
+void* static_scratch_on_current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (g_static_scratch_addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_bwd_static_scratch) != cudaSuccess) return nullptr;
+    g_static_scratch_addr[dev] = ptr;
+  }
+  return g_static_scratch_addr[dev];
+}
+}  // namespace
+
+extern "C" {
+
+sqa_status_t sqa_attn_bwd_static(const void* q, const void* k, const void* v, const void* out, sqa_dtype_t o_dtype,
+                                 const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                                 sqa_dtype_t grad_dtype, int B, int N, int H_q, int H_kv, int d_head, int causal,
+                                 float scale, void* stream) {
+  const size_t need = sqa_attn_bwd_workspace_size(B, N, H_q, H_kv, d_head);
+  if (need == 0) return SQA_ERR_INVALID_ARG;
+  if (need > SQA_BWD_STATIC_SCRATCH_BYTES) return SQA_ERR_UNSUPPORTED;
+  void* scratch = static_scratch_on_current_device();
+  if (scratch == nullptr) return SQA_ERR_CUDA;
+  return sqa_attn_bwd(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B, N, H_q, H_kv, d_head, causal,
+                      scale, scratch, SQA_BWD_STATIC_SCRATCH_BYTES, stream);
+}
+
 sqa_status_t sqa_proj(const void* x, const void* w, const float* bias, void* y, sqa_dtype_t y_dtype, int M, int K,
                       int Nout, void* stream) {
   if (!x || !w || !y) return SQA_ERR_INVALID_ARG;
