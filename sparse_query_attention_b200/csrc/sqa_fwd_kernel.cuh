@@ -65,6 +65,11 @@ struct FwdParams {
 };
 
 constexpr int kFwdThreads = 384;
+constexpr int kFwdRegsLaunch = 168;  // per thread at launch (launch bounds 384 x 1)
+constexpr int kFwdRegsLow = 88;      // producer / MMA warpgroup after reallocation
+constexpr int kFwdRegsHigh = 208;    // each softmax warpgroup after reallocation
+static_assert(kFwdRegsLow * 128 + kFwdRegsHigh * 256 <= kFwdRegsLaunch * kFwdThreads,
+              "register split exceeds the launch pool");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only past 2^8 growth
 
 template <int D>
@@ -77,7 +82,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   __shared__ __align__(8) uint64_t slot_full[C::kSlots];
   __shared__ __align__(8) uint64_t slot_empty[C::kSlots];
   __shared__ __align__(8) uint64_t s_full[2];
-  __shared__ __align__(8) uint64_t p_ready[2];
+  __shared__ __align__(8) uint64_t p_ready[2][2];  // [tile][half of the keys]
   __shared__ __align__(8) uint64_t o_done[2];
   __shared__ __align__(8) uint64_t mma_done;
   __shared__ uint32_t tmem_base_sh;
@@ -119,7 +124,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_ready[t], 4);  // one arrival per softmax warp
+      mbar_init(&p_ready[t][0], 4);  // one arrival per softmax warp
+      mbar_init(&p_ready[t][1], 4);
       mbar_init(&o_done[t], 1);
     }
     mbar_init(&mma_done, 1);
@@ -139,7 +145,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-
+  // Registers: the block launches with 384 x 168; the producer/MMA
+  // warpgroup needs few, the two softmax warpgroups hold a 128-column score
+  // row each: 88 * 128 + 208 * 256 = 168 * 384.  Each warpgroup reallocates
+  // at the top of its own branch, so the register allocator sees which limit
+  // governs which code.
+  if (warp < 4) {
+  regs_dealloc<kFwdRegsLow>();
   if (warp == 0) {
     // ======================= TMA producer =================================
     if (lane == 0) {
@@ -188,12 +200,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           mma_ss(tmem + col_s[t], a, bd, idesc_s, kk > 0);
         }
       };
-      auto issue_pv = [&](int t, int slot, bool acc) {
+      // Four 16-key MMAs over keys [16 k0, 16 k0 + 64).
+      auto issue_pv = [&](int t, int slot, bool acc, int k0) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // 16 keys per MMA
+        for (int kk = k0; kk < k0 + 4; ++kk) {
           const uint64_t bd = smem_desc(ring_addr + slot * C::kTileBytes + kk * 16 * C::kRowBytes, C::kChunkBytes,
                                         8 * C::kRowBytes, C::kSwizzle);
-          mma_ts(tmem + col_o[t], tmem + col_s[t] + kk * 8, bd, idesc_o, (acc || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + col_o[t], tmem + col_s[t] + kk * 8, bd, idesc_o, (acc || kk > k0) ? 1u : 0u);
         }
       };
 
@@ -215,19 +228,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (!mbar_wait(&slot_full[vs], (vpos / C::kSlots) & 1, &abort_flag)) break;
         const bool more = i + 1 < n_steps;
         if (more && !mbar_wait(&slot_full[ks], (kpos / C::kSlots) & 1, &abort_flag)) break;
-        // tile 0: O_0 += P_0 V_i, then S_0 = Q_0 K_{i+1}^T
-        if (!mbar_wait(&p_ready[0], i & 1, &abort_flag)) break;
+        // tile 0: O_0 += P_0 V_i (keys 0-63 as soon as that half of P is
+        // in TMEM, then keys 64-127), then S_0 = Q_0 K_{i+1}^T
+        if (!mbar_wait(&p_ready[0][0], i & 1, &abort_flag)) break;
         tc_fence_after();
-        issue_pv(0, vs, i > 0);
+        issue_pv(0, vs, i > 0, 0);
+        if (!mbar_wait(&p_ready[0][1], i & 1, &abort_flag)) break;
+        tc_fence_after();
+        issue_pv(0, vs, true, 4);
         mma_commit(&o_done[0]);
         if (more) {
           issue_s(0, ks);
           mma_commit(&s_full[0]);
         }
         // tile 1
-        if (!mbar_wait(&p_ready[1], i & 1, &abort_flag)) break;
+        if (!mbar_wait(&p_ready[1][0], i & 1, &abort_flag)) break;
         tc_fence_after();
-        issue_pv(1, vs, i > 0);
+        issue_pv(1, vs, i > 0, 0);
+        if (!mbar_wait(&p_ready[1][1], i & 1, &abort_flag)) break;
+        tc_fence_after();
+        issue_pv(1, vs, true, 4);
         mma_commit(&o_done[1]);
         mma_commit(&slot_empty[vs]);
         if (more) {
@@ -239,7 +259,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       (void)kslot;
       mma_commit(&mma_done);
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    regs_alloc<kFwdRegsHigh>();
     // ======================= softmax + epilogue ===========================
     const int t = (warp - 4) >> 2;  // tile
     const int wq = warp & 3;        // TMEM lane quarter
@@ -270,21 +292,46 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tmem_wait_ld();
       float s[128];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]) * sl2;
+      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
       // Masking: keys past N, and keys after the query token when causal.
+      // Unmasked tiles (the common case) keep raw scores: the row max is
+      // taken on them and the scale is folded into the exponent's FFMA.
+      // Masked tiles are scaled first and get -inf where masked.
       const int key0 = i * 128;
       const bool need_mask = (key0 + 128 > p.N) || (p.causal && key0 + 127 > tile_tok_min) || i >= n_kv[t];
+      float mult = sl2;  // exponent argument = s * mult - m
       if (need_mask) {
         int lim = p.N - key0;                                   // keys [0, lim) are < N
         if (p.causal) lim = min(lim, tok - key0 + 1);           // keys <= tok
         if (i >= n_kv[t]) lim = 0;
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= lim) s[c] = -INFINITY;
+        for (int c = 0; c < 128; ++c) s[c] = c < lim ? s[c] * sl2 : -INFINITY;
+        mult = 1.f;
       }
-      float mx = s[0];
+      // Row max (row min for a negative scale on raw scores): eight
+      // independent 3-input chains, then a short merge.  The sign test is a
+      // uniform branch around whole loops, not a select per element.
+      const bool use_min = !need_mask && sl2 < 0.f;
+      float acc8[8];
+      float ext;
+      if (use_min) {
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+        for (int k = 0; k < 8; ++k) acc8[k] = fminf(s[k], s[k + 8]);
+#pragma unroll
+        for (int c = 16; c < 128; c += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc8[k] = fmin3(acc8[k], s[c + k], s[c + 8 + k]);
+        ext = fmin3(fmin3(acc8[0], acc8[1], acc8[2]), fmin3(acc8[3], acc8[4], acc8[5]), fminf(acc8[6], acc8[7]));
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc8[k] = fmaxf(s[k], s[k + 8]);
+#pragma unroll
+        for (int c = 16; c < 128; c += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc8[k] = fmax3(acc8[k], s[c + k], s[c + 8 + k]);
+        ext = fmax3(fmax3(acc8[0], acc8[1], acc8[2]), fmax3(acc8[3], acc8[4], acc8[5]), fmaxf(acc8[6], acc8[7]));
+      }
+      const float mx = ext * mult;
       const float m_new = fmaxf(m_used, mx);
       // Rescale only when the running max grew by more than the threshold
       // (or on the first finite max); otherwise keep exponentiating against
@@ -314,22 +361,42 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         m_used = m_new;
       }
       const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
-      float rs = 0.f;
-      uint32_t pk[64];
+      // P = 2^(s * mult - m): one packed FFMA per pair; every fourth pair on
+      // the FMA pipe (polynomial), the rest on the MUFU; row sum in four
+      // packed accumulators.  Keys 0-63 are stored and handed to the MMA
+      // warp first, so the first half of O += P V runs while keys 64-127
+      // are exponentiated.
+      const uint64_t mult2 = f2_pack(mult, mult);
+      const uint64_t negm2 = f2_pack(-m_sub, -m_sub);
+      uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2_approx(s[2 * c] - m_sub);
-        const float p1 = ex2_approx(s[2 * c + 1] - m_sub);
-        rs += p0 + p1;
-        pk[c] = pack_bf16x2(p0, p1);
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int cc = 0; cc < 32; ++cc) {
+          const int c = half * 32 + cc;
+          float x0, x1, p0, p1;
+          f2_unpack(f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), mult2, negm2), x0, x1);
+          if ((c & 3) == 3) {
+            exp2_poly_pair(x0, x1, p0, p1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          sum2[c & 3] = f2_add(sum2[c & 3], f2_pack(p0, p1));
+          pk[cc] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(s_addr + half * 32, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_ready[t][half]);
       }
-      l_sum += rs;
-      tmem_st32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_ready[t]);
+      {
+        float a0, a1;
+        f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), a0, a1);
+        l_sum += a0 + a1;
+      }
     }
     // Epilogue: O / l and LSE once the last PV of this tile has landed.
     if (ok) ok = mbar_wait(&o_done[t], (my_steps - 1) & 1, &abort_flag);
