@@ -32,8 +32,9 @@
 namespace sqa {
 
 // ---------------------------------------------------------------------------
-// Preprocess: D[b,h,t] = sum_c dO[b,t,h,c] O[b,t,h,c]; L2[b,h,t] = LSE * log2 e.
-// Workspace rows are padded to n_pad tokens (multiple of 128) with zeros.
+// Preprocess: D[b,h,t] = sum_c dO[b,t,h,c] O[b,t,h,c]; L2[b,h,t] = LSE * log2 e,
+// both stored negated.  Workspace rows are padded to n_pad tokens (multiple of
+// 128) with zeros.
 // One warp per (b, h, t) of the padded space.
 // ---------------------------------------------------------------------------
 template <int D>
@@ -60,9 +61,9 @@ __global__ void bwd_prep_kernel(const void* __restrict__ o, int o_bf16, const __
     for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
     l2 = lse[bh * N + t] * 1.4426950408889634f;
   }
-  if (lane == 0) {
-    dsum[idx] = acc;
-    lse2[idx] = l2;
+  if (lane == 0) {  // stored negated: the kernels add them in packed FFMA/FADD
+    dsum[idx] = -acc;
+    lse2[idx] = -l2;
   }
 }
 
@@ -122,6 +123,11 @@ struct BwdParams {
 };
 
 constexpr int kBwdThreads = 384;
+// Register split after launch (384 x 168): producer/MMA warpgroup 88, the two
+// softmax-gradient warpgroups 208 each; 88 * 128 + 208 * 256 = 168 * 384.
+constexpr int kBwdRegsLow = 88;
+constexpr int kBwdRegsHigh = 208;
+static_assert(kBwdRegsLow * 128 + kBwdRegsHigh * 256 <= 168 * kBwdThreads, "register split exceeds the launch pool");
 
 // ===========================================================================
 // dK / dV
@@ -198,6 +204,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
+  if (warp < 4) {
+  regs_dealloc<kBwdRegsLow>();
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
@@ -273,7 +281,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       mma_commit(&mma_done);
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    regs_alloc<kBwdRegsHigh>();
     // ---------------- softmax-gradient warps ----------------
     const int grp = (warp - 4) >> 2;  // handles steps s with s % 2 == grp
     const int wq = warp & 3;
@@ -298,25 +308,48 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float* dd = reinterpret_cast<const float*>(stat + 256);
       const int q0 = (qs_begin + s % per_head) * 64;
       // Query column c (token q0 + c) contributes iff q0 + c < N and, when
-      // causal, q0 + c >= u.
-      int lo = p.causal ? u - q0 : 0;          // first allowed column
-      const int hi = p.N - q0;                 // columns [0, hi) are < N
+      // causal, q0 + c >= u.  Full tiles skip the per-element test.
+      const int lo = p.causal ? u - q0 : 0;  // first allowed column
+      const int hi = p.N - q0;               // columns [0, hi) are < N
+      const bool full = __all_sync(0xffffffffu, lo <= 0 && hi >= 64);
       tmem_wait_ld();
       uint32_t pk[32], dk[32];
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
+      // P = 2^(s sl2 - L2), dS = P (dP - D), two columns per packed op; the
+      // workspace holds -L2 and -D.  A quarter of the exponentials run as
+      // the FMA-pipe polynomial.
+      auto body = [&](auto masked) {
 #pragma unroll
-      for (int c2 = 0; c2 < 32; ++c2) {
-        float pv[2], dsv[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int c = 2 * c2 + e;
-          const bool keep = c >= lo && c < hi;
-          const float pr = ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, -l2[c]));
-          pv[e] = keep ? pr : 0.f;
-          dsv[e] = keep ? pr * (__uint_as_float(dr[c]) - dd[c]) : 0.f;
+        for (int c2 = 0; c2 < 32; ++c2) {
+          const int c = 2 * c2;
+          const float2 nl = *reinterpret_cast<const float2*>(l2 + c);
+          const float2 nd = *reinterpret_cast<const float2*>(dd + c);
+          float x0, x1, p0, p1, d0, d1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, f2_pack(nl.x, nl.y)),
+                    x0, x1);
+          if ((c2 & 3) == 3) {
+            exp2_poly_pair(x0, x1, p0, p1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          const uint64_t t = f2_add(f2_pack(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])), f2_pack(nd.x, nd.y));
+          f2_unpack(f2_mul(f2_pack(p0, p1), t), d0, d1);
+          if constexpr (decltype(masked)::value) {
+            const bool k0 = c >= lo && c < hi, k1 = c + 1 >= lo && c + 1 < hi;
+            p0 = k0 ? p0 : 0.f;
+            d0 = k0 ? d0 : 0.f;
+            p1 = k1 ? p1 : 0.f;
+            d1 = k1 ? d1 : 0.f;
+          }
+          pk[c2] = pack_bf16x2(p0, p1);
+          dk[c2] = pack_bf16x2(d0, d1);
         }
-        pk[c2] = pack_bf16x2(pv[0], pv[1]);
-        dk[c2] = pack_bf16x2(dsv[0], dsv[1]);
-      }
+      };
+      if (full)
+        body(BoolC<false>{});
+      else
+        body(BoolC<true>{});
       tmem_st32(lane_base + C::col_s(grp), pk);
       tmem_st32(lane_base + C::col_dp(grp), dk);
       tmem_wait_st();
@@ -430,6 +463,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
+  if (warp < 4) {
+  regs_dealloc<kBwdRegsLow>();
   if (warp == 0) {
     if (lane == 0) {
       mbar_arrive_expect_tx(&q_full, 2 * QT::kBytes);
@@ -494,7 +529,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       mma_commit(&mma_done);
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    regs_alloc<kBwdRegsHigh>();
     const int grp = (warp - 4) >> 2;
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
@@ -503,8 +540,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const float sl2 = p.scale_log2;
     const size_t stat = (static_cast<size_t>(b) * p.H_q + head) * p.n_pad + tok;  // tok < n_pad
-    const float l2 = p.lse2[stat];
-    const float dd = p.dsum[stat];
+    const float nl2 = p.lse2[stat];  // -LSE * log2(e)
+    const float ndd = p.dsum[stat];  // -D
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
+    const uint64_t nl2x2 = f2_pack(nl2, nl2);
+    const uint64_t ndd2 = f2_pack(ndd, ndd);
     bool ok = true;
     for (int s = grp; s < n_steps; s += 2) {
       if (!mbar_wait(&s_full[grp], (s >> 1) & 1, &abort_flag)) {
@@ -520,19 +560,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int kbase = s * 64;
       int hi = p.N - kbase;                        // keys [0, hi) are < N
       if (p.causal) hi = min(hi, tok - kbase + 1);  // keys <= tok
+      const bool full = __all_sync(0xffffffffu, hi >= 64);
       tmem_wait_ld();
       uint32_t dk[32];
+      // dS = 2^(s sl2 - L2) (dP - D) with the row's -L2 and -D (nl2, ndd),
+      // two keys per packed op, a quarter of the exponentials as the
+      // FMA-pipe polynomial; full tiles skip the per-element key test.
+      auto body = [&](auto masked) {
 #pragma unroll
-      for (int c2 = 0; c2 < 32; ++c2) {
-        float dsv[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int c = 2 * c2 + e;
-          const float pr = ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, -l2));
-          dsv[e] = c < hi ? pr * (__uint_as_float(dr[c]) - dd) : 0.f;
+        for (int c2 = 0; c2 < 32; ++c2) {
+          const int c = 2 * c2;
+          float x0, x1, p0, p1, d0, d1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, nl2x2), x0, x1);
+          if ((c2 & 3) == 3) {
+            exp2_poly_pair(x0, x1, p0, p1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          const uint64_t t = f2_add(f2_pack(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])), ndd2);
+          f2_unpack(f2_mul(f2_pack(p0, p1), t), d0, d1);
+          if constexpr (decltype(masked)::value) {
+            d0 = c < hi ? d0 : 0.f;
+            d1 = c + 1 < hi ? d1 : 0.f;
+          }
+          dk[c2] = pack_bf16x2(d0, d1);
         }
-        dk[c2] = pack_bf16x2(dsv[0], dsv[1]);
-      }
+      };
+      if (full)
+        body(BoolC<false>{});
+      else
+        body(BoolC<true>{});
       tmem_st32(lane_base + C::col_s(grp), dk);
       tmem_wait_st();
       tc_fence_before();
