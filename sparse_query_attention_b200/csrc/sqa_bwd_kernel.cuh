@@ -96,17 +96,16 @@ struct TileGeo {
   static constexpr uint32_t kSwizzle = kRowBytes == 128 ? kSw128 : (kRowBytes == 64 ? kSw64 : kSw32);
   static constexpr uint32_t kSbo = 8 * kRowBytes;
 
-  // K-major operand (rows = M or N, K = D): descriptor for the 16-wide K step kk.
-  __device__ static uint64_t kmajor(uint32_t base, int kk) {
-    const int c = (kk * 16) / kRowElems;
-    const uint32_t off = c * kChunkBytes + ((kk * 16) % kRowElems) * 2;
-    return smem_desc(base + off, 16, kSbo, kSwizzle);
+  // K-major operand (rows = M or N, K = D): base descriptor of a tile, and
+  // the byte offset of the 16-wide K step kk within it.
+  __device__ static uint64_t kmajor_base(uint32_t base) { return smem_desc(base, 16, kSbo, kSwizzle); }
+  __host__ __device__ static constexpr uint32_t kmajor_off(int kk) {
+    return ((kk * 16) / kRowElems) * kChunkBytes + ((kk * 16) % kRowElems) * 2;
   }
-  // MN-major operand (N = D along the row, K = rows): descriptor for rows
-  // [16 kk, 16 kk + 16).
-  __device__ static uint64_t mnmajor(uint32_t base, int kk) {
-    return smem_desc(base + kk * 16 * kRowBytes, kChunkBytes, kSbo, kSwizzle);
-  }
+  // MN-major operand (N = D along the row, K = rows): base descriptor, and
+  // the byte offset of rows [16 kk, 16 kk + 16).
+  __device__ static uint64_t mnmajor_base(uint32_t base) { return smem_desc(base, kChunkBytes, kSbo, kSwizzle); }
+  __host__ __device__ static constexpr uint32_t mnmajor_off(int kk) { return kk * 16 * kRowBytes; }
 };
 
 struct BwdParams {
@@ -123,10 +122,10 @@ struct BwdParams {
 };
 
 constexpr int kBwdThreads = 384;
-// Register split after launch (384 x 168): producer/MMA warpgroup 88, the two
-// softmax-gradient warpgroups 208 each; 88 * 128 + 208 * 256 = 168 * 384.
-constexpr int kBwdRegsLow = 88;
-constexpr int kBwdRegsHigh = 208;
+// Register split after launch (384 x 168): producer/MMA warpgroup 104, the two
+// softmax-gradient warpgroups 200 each; 104 * 128 + 200 * 256 = 168 * 384.
+constexpr int kBwdRegsLow = 104;
+constexpr int kBwdRegsHigh = 200;
 static_assert(kBwdRegsLow * 128 + kBwdRegsHigh * 256 <= 168 * kBwdThreads, "register split exceeds the launch pool");
 
 // ===========================================================================
@@ -238,17 +237,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // ---------------- MMA issuer ----------------
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);  // M=128 keys, N=64 queries
       constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, 0, 1);   // M=128 keys, N=D, B MN-major
-      const uint32_t k_addr = smem_addr(k_smem), v_addr = smem_addr(v_smem);
-      const uint32_t st_addr = smem_addr(stages);
+      // Descriptors are built once; every MMA only adds a constant offset
+      // (a single-thread dependent chain of descriptor arithmetic per MMA
+      // would take longer to issue than the MMA takes to run).
+      const uint64_t k_kd = KV::kmajor_base(smem_addr(k_smem));
+      const uint64_t v_kd = KV::kmajor_base(smem_addr(v_smem));
+      const uint64_t st_kd = QT::kmajor_base(smem_addr(stages));
+      const uint64_t st_mn = QT::mnmajor_base(smem_addr(stages));
       auto issue_scores = [&](int s) {
         const int buf = s & 1;
-        const uint32_t qa = st_addr + (s % C::kStages) * C::kStageBytes;
+        const uint64_t q_kd = desc_advance(st_kd, (s % C::kStages) * C::kStageBytes);
+        const uint64_t do_kd = desc_advance(q_kd, QT::kBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + C::col_s(buf), KV::kmajor(k_addr, kk), QT::kmajor(qa, kk), idesc_s, kk > 0);
+          mma_ss(tmem + C::col_s(buf), desc_advance(k_kd, KV::kmajor_off(kk)), desc_advance(q_kd, QT::kmajor_off(kk)),
+                 idesc_s, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + C::col_dp(buf), KV::kmajor(v_addr, kk), QT::kmajor(qa + QT::kBytes, kk), idesc_s, kk > 0);
+          mma_ss(tmem + C::col_dp(buf), desc_advance(v_kd, KV::kmajor_off(kk)),
+                 desc_advance(do_kd, QT::kmajor_off(kk)), idesc_s, kk > 0);
         mma_commit(&s_full[buf]);
       };
       bool ok = mbar_wait(&kv_full, 0, &abort_flag);
@@ -263,14 +270,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int buf = s & 1;
         if (!mbar_wait(&p_ready[buf], (s >> 1) & 1, &abort_flag)) break;
         tc_fence_after();
-        const uint32_t qa = st_addr + (s % C::kStages) * C::kStageBytes;
+        const uint64_t q_mn = desc_advance(st_mn, (s % C::kStages) * C::kStageBytes);
+        const uint64_t do_mn = desc_advance(q_mn, QT::kBytes);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // 64 query rows = 4 x K16
-          mma_ts(tmem + C::kColDV, tmem + C::col_s(buf) + kk * 8, QT::mnmajor(qa + QT::kBytes, kk), idesc_g,
+          mma_ts(tmem + C::kColDV, tmem + C::col_s(buf) + kk * 8, desc_advance(do_mn, QT::mnmajor_off(kk)), idesc_g,
                  (s > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + C::kColDK, tmem + C::col_dp(buf) + kk * 8, QT::mnmajor(qa, kk), idesc_g,
+          mma_ts(tmem + C::kColDK, tmem + C::col_dp(buf) + kk * 8, desc_advance(q_mn, QT::mnmajor_off(kk)), idesc_g,
                  (s > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&st_empty[s % C::kStages]);
         if (s + 2 < n_steps) {
@@ -490,17 +498,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);  // M=128 rows, N=64 keys
       constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, 0, 1);   // M=128 rows, N=D, B MN-major
-      const uint32_t q_addr = smem_addr(q_smem), do_addr = smem_addr(do_smem);
-      const uint32_t st_addr = smem_addr(stages);
+      // Descriptors built once; each MMA adds a constant offset.
+      const uint64_t q_kd = QT::kmajor_base(smem_addr(q_smem));
+      const uint64_t do_kd = QT::kmajor_base(smem_addr(do_smem));
+      const uint64_t st_kd = KS::kmajor_base(smem_addr(stages));
+      const uint64_t st_mn = KS::mnmajor_base(smem_addr(stages));
       auto issue_scores = [&](int s) {
         const int buf = s & 1;
-        const uint32_t ka = st_addr + (s % C::kStages) * C::kStageBytes;
+        const uint64_t k_kd = desc_advance(st_kd, (s % C::kStages) * C::kStageBytes);
+        const uint64_t v_kd = desc_advance(k_kd, KS::kBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + C::col_s(buf), QT::kmajor(q_addr, kk), KS::kmajor(ka, kk), idesc_s, kk > 0);
+          mma_ss(tmem + C::col_s(buf), desc_advance(q_kd, QT::kmajor_off(kk)), desc_advance(k_kd, KS::kmajor_off(kk)),
+                 idesc_s, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + C::col_dp(buf), QT::kmajor(do_addr, kk), KS::kmajor(ka + KS::kBytes, kk), idesc_s, kk > 0);
+          mma_ss(tmem + C::col_dp(buf), desc_advance(do_kd, QT::kmajor_off(kk)),
+                 desc_advance(v_kd, KS::kmajor_off(kk)), idesc_s, kk > 0);
         mma_commit(&s_full[buf]);
       };
       bool ok = mbar_wait(&q_full, 0, &abort_flag);
@@ -515,10 +529,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int buf = s & 1;
         if (!mbar_wait(&p_ready[buf], (s >> 1) & 1, &abort_flag)) break;
         tc_fence_after();
-        const uint32_t ka = st_addr + (s % C::kStages) * C::kStageBytes;
+        const uint64_t k_mn = desc_advance(st_mn, (s % C::kStages) * C::kStageBytes);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // 64 keys = 4 x K16
-          mma_ts(tmem + C::kColDQ, tmem + C::col_s(buf) + kk * 8, KS::mnmajor(ka, kk), idesc_g,
+          mma_ts(tmem + C::kColDQ, tmem + C::col_s(buf) + kk * 8, desc_advance(k_mn, KS::mnmajor_off(kk)), idesc_g,
                  (s > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&st_empty[s % C::kStages]);
         if (s + 2 < n_steps) {

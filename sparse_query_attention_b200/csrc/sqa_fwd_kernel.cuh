@@ -185,29 +185,30 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t q_addr = smem_addr(q_smem);
-      const uint32_t ring_addr = smem_addr(ring);
       const uint32_t col_s[2] = {C::kColS0, C::kColS1};
       const uint32_t col_o[2] = {C::kColO0, C::kColO1};
+      // Descriptors are built once; each MMA adds a constant offset.
+      const uint64_t q_kd = smem_desc(smem_addr(q_smem), 16, 8 * C::kRowBytes, C::kSwizzle);
+      const uint64_t ring_kd = smem_desc(smem_addr(ring), 16, 8 * C::kRowBytes, C::kSwizzle);
+      const uint64_t ring_mn = smem_desc(smem_addr(ring), C::kChunkBytes, 8 * C::kRowBytes, C::kSwizzle);
 
       auto issue_s = [&](int t, int slot) {
+        const uint64_t a0 = desc_advance(q_kd, t * C::kTileBytes);
+        const uint64_t b0 = desc_advance(ring_kd, slot * C::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const int c = (kk * 16) / C::kRowElems;
-          const uint32_t off = c * C::kChunkBytes + ((kk * 16) % C::kRowElems) * 2;
-          const uint64_t a = smem_desc(q_addr + t * C::kTileBytes + off, 16, 8 * C::kRowBytes, C::kSwizzle);
-          const uint64_t bd = smem_desc(ring_addr + slot * C::kTileBytes + off, 16, 8 * C::kRowBytes, C::kSwizzle);
-          mma_ss(tmem + col_s[t], a, bd, idesc_s, kk > 0);
+          constexpr int kPerChunk = C::kRowElems / 16;
+          const uint32_t off = (kk / kPerChunk) * C::kChunkBytes + (kk % kPerChunk) * 32;
+          mma_ss(tmem + col_s[t], desc_advance(a0, off), desc_advance(b0, off), idesc_s, kk > 0);
         }
       };
       // Four 16-key MMAs over keys [16 k0, 16 k0 + 64).
       auto issue_pv = [&](int t, int slot, bool acc, int k0) {
+        const uint64_t b0 = desc_advance(ring_mn, slot * C::kTileBytes);
 #pragma unroll
-        for (int kk = k0; kk < k0 + 4; ++kk) {
-          const uint64_t bd = smem_desc(ring_addr + slot * C::kTileBytes + kk * 16 * C::kRowBytes, C::kChunkBytes,
-                                        8 * C::kRowBytes, C::kSwizzle);
-          mma_ts(tmem + col_o[t], tmem + col_s[t] + kk * 8, bd, idesc_o, (acc || kk > k0) ? 1u : 0u);
-        }
+        for (int kk = k0; kk < k0 + 4; ++kk)
+          mma_ts(tmem + col_o[t], tmem + col_s[t] + kk * 8, desc_advance(b0, kk * 16 * C::kRowBytes), idesc_o,
+                 (acc || kk > k0) ? 1u : 0u);
       };
 
       bool ok = mbar_wait(&q_full, 0, &abort_flag);
