@@ -23,8 +23,10 @@
 //   bwd_dq_kernel     Q-outer: one CTA per 128 packed query rows (as in the
 //                     forward); per 64-key sub-tile: S = Q K^T, dP = dO V^T,
 //                     dS in TMEM, dQ += dS K.
-// Score tiles are 64 wide and double-buffered in TMEM so that the softmax of
-// one buffer overlaps the tensor-core work on the other.
+// Score tiles are 64 wide and held in two or three TMEM buffers (three where
+// the columns allow): the scores of step s + buffers are computed as soon as
+// step s's products have read its buffer, so the softmax warps, which take
+// steps in turn, find their scores ready.
 #pragma once
 
 #include "sqa_ptx.cuh"
@@ -135,14 +137,17 @@ template <int D>
 struct DkdvCfg {
   using KV = TileGeo<D, 128>;  // resident K and V tiles
   using QT = TileGeo<D, 64>;   // streamed Q / dO sub-tiles
-  static constexpr int kStages = 4;
+  static constexpr int kStages = D == 128 ? 4 : 6;
   static constexpr int kStatBytes = 1024;                        // LSE2 (256 B) + D (256 B), 1 KB aligned
   static constexpr int kStageBytes = 2 * QT::kBytes + kStatBytes;  // Q, dO, stats
   static constexpr int kSmemBytes = 2 * KV::kBytes + kStages * kStageBytes + 1024;
+  // Score buffers in TMEM: three when they fit next to dV and dK (d <= 64).
+  static constexpr int kBufs = D <= 64 ? 3 : 2;
   // TMEM columns: S^T/P^T and dP^T/dS^T of buffer b, then dV and dK.
   __device__ static constexpr uint32_t col_s(int b) { return 128u * b; }
   __device__ static constexpr uint32_t col_dp(int b) { return 64u + 128u * b; }
-  static constexpr uint32_t kColDV = 256, kColDK = 256 + D;
+  static constexpr uint32_t kColDV = 128 * kBufs, kColDK = 128 * kBufs + D;
+  static_assert(kColDK + D <= 512, "TMEM columns");
 };
 
 template <int D, typename GradT>
@@ -158,8 +163,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __shared__ __align__(8) uint64_t kv_full;
   __shared__ __align__(8) uint64_t st_full[C::kStages];
   __shared__ __align__(8) uint64_t st_empty[C::kStages];
-  __shared__ __align__(8) uint64_t s_full[2];
-  __shared__ __align__(8) uint64_t p_ready[2];
+  __shared__ __align__(8) uint64_t s_full[C::kBufs];
+  __shared__ __align__(8) uint64_t p_ready[C::kBufs];
   __shared__ __align__(8) uint64_t mma_done;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -186,7 +191,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&st_full[s], 1);
       mbar_init(&st_empty[s], 1);
     }
-    for (int t = 0; t < 2; ++t) {
+    for (int t = 0; t < C::kBufs; ++t) {
       mbar_init(&s_full[t], 1);
       mbar_init(&p_ready[t], 4);
     }
@@ -233,8 +238,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int l = max(0, s - C::kStages); l < s; ++l) mbar_drain(&st_full[l % C::kStages], (l / C::kStages) & 1);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
+    {
+      // ---------------- MMA issuer: whole warp, lane 0 issues ----------------
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);  // M=128 keys, N=64 queries
       constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, 0, 1);   // M=128 keys, N=D, B MN-major
       // Descriptors are built once; every MMA only adds a constant offset
@@ -245,21 +250,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t st_kd = QT::kmajor_base(smem_addr(stages));
       const uint64_t st_mn = QT::mnmajor_base(smem_addr(stages));
       auto issue_scores = [&](int s) {
-        const int buf = s & 1;
+        const int buf = s % C::kBufs;
         const uint64_t q_kd = desc_advance(st_kd, (s % C::kStages) * C::kStageBytes);
         const uint64_t do_kd = desc_advance(q_kd, QT::kBytes);
+        // S^T and dP^T accumulate separately: alternating their K steps keeps
+        // two independent MMA chains in flight.
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + C::col_s(buf), desc_advance(k_kd, KV::kmajor_off(kk)), desc_advance(q_kd, QT::kmajor_off(kk)),
+        for (int kk = 0; kk < D / 16; ++kk) {
+          mma_ss_w(tmem + C::col_s(buf), desc_advance(k_kd, KV::kmajor_off(kk)), desc_advance(q_kd, QT::kmajor_off(kk)),
                  idesc_s, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + C::col_dp(buf), desc_advance(v_kd, KV::kmajor_off(kk)),
+          mma_ss_w(tmem + C::col_dp(buf), desc_advance(v_kd, KV::kmajor_off(kk)),
                  desc_advance(do_kd, QT::kmajor_off(kk)), idesc_s, kk > 0);
-        mma_commit(&s_full[buf]);
+        }
+        mma_commit_w(&s_full[buf]);
       };
       bool ok = mbar_wait(&kv_full, 0, &abort_flag);
-      for (int s = 0; s < 2 && s < n_steps && ok; ++s) {
+      for (int s = 0; s < C::kBufs && s < n_steps && ok; ++s) {
         ok = mbar_wait(&st_full[s % C::kStages], (s / C::kStages) & 1, &abort_flag);
         if (ok) {
           tc_fence_after();
@@ -267,27 +273,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
       for (int s = 0; s < n_steps && ok; ++s) {
-        const int buf = s & 1;
-        if (!mbar_wait(&p_ready[buf], (s >> 1) & 1, &abort_flag)) break;
+        const int buf = s % C::kBufs;
+        if (!mbar_wait(&p_ready[buf], (s / C::kBufs) & 1, &abort_flag)) break;
         tc_fence_after();
         const uint64_t q_mn = desc_advance(st_mn, (s % C::kStages) * C::kStageBytes);
         const uint64_t do_mn = desc_advance(q_mn, QT::kBytes);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)  // 64 query rows = 4 x K16
-          mma_ts(tmem + C::kColDV, tmem + C::col_s(buf) + kk * 8, desc_advance(do_mn, QT::mnmajor_off(kk)), idesc_g,
+        for (int kk = 0; kk < 4; ++kk) {  // 64 query rows = 4 x K16; dV and dK chains alternate
+          mma_ts_w(tmem + C::kColDV, tmem + C::col_s(buf) + kk * 8, desc_advance(do_mn, QT::mnmajor_off(kk)), idesc_g,
                  (s > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + C::kColDK, tmem + C::col_dp(buf) + kk * 8, desc_advance(q_mn, QT::mnmajor_off(kk)), idesc_g,
+          mma_ts_w(tmem + C::kColDK, tmem + C::col_dp(buf) + kk * 8, desc_advance(q_mn, QT::mnmajor_off(kk)), idesc_g,
                  (s > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&st_empty[s % C::kStages]);
-        if (s + 2 < n_steps) {
-          if (!mbar_wait(&st_full[(s + 2) % C::kStages], ((s + 2) / C::kStages) & 1, &abort_flag)) break;
+        }
+        mma_commit_w(&st_empty[s % C::kStages]);
+        if (s + C::kBufs < n_steps) {  // the next scores into the buffer just read
+          const int s2 = s + C::kBufs;
+          if (!mbar_wait(&st_full[s2 % C::kStages], (s2 / C::kStages) & 1, &abort_flag)) break;
           tc_fence_after();
-          issue_scores(s + 2);
+          issue_scores(s2);
         }
       }
-      mma_commit(&mma_done);
+      mma_commit_w(&mma_done);
     }
   }
   } else {
@@ -301,16 +307,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float sl2 = p.scale_log2;
     bool ok = true;
     for (int s = grp; s < n_steps; s += 2) {
-      if (!mbar_wait(&s_full[grp], (s >> 1) & 1, &abort_flag)) {
+      const int buf = s % C::kBufs;
+      if (!mbar_wait(&s_full[buf], (s / C::kBufs) & 1, &abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
       uint32_t sr[64], dr[64];
-      tmem_ld32(lane_base + C::col_s(grp), *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(lane_base + C::col_s(grp) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld32(lane_base + C::col_dp(grp), *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
-      tmem_ld32(lane_base + C::col_dp(grp) + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+      tmem_ld32(lane_base + C::col_s(buf), *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(lane_base + C::col_s(buf) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(lane_base + C::col_dp(buf), *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+      tmem_ld32(lane_base + C::col_dp(buf) + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
       const uint8_t* stat = stages + (s % C::kStages) * C::kStageBytes + 2 * QT::kBytes;
       const float* l2 = reinterpret_cast<const float*>(stat);
       const float* dd = reinterpret_cast<const float*>(stat + 256);
@@ -358,12 +365,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         body(BoolC<false>{});
       else
         body(BoolC<true>{});
-      tmem_st32(lane_base + C::col_s(grp), pk);
-      tmem_st32(lane_base + C::col_dp(grp), dk);
+      tmem_st32(lane_base + C::col_s(buf), pk);
+      tmem_st32(lane_base + C::col_dp(buf), dk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_ready[grp]);
+      if (lane == 0) mbar_arrive(&p_ready[buf]);
     }
     // ---------------- epilogue: group 0 writes dV, group 1 writes dK --------
     if (ok) ok = mbar_wait(&mma_done, 0, &abort_flag);
@@ -404,13 +411,15 @@ template <int D>
 struct DqCfg {
   using QT = TileGeo<D, 128>;  // resident Q and dO tiles (packed rows)
   using KS = TileGeo<D, 64>;   // streamed K / V sub-tiles
-  static constexpr int kStages = 4;
+  static constexpr int kStages = D == 128 ? 4 : 6;
   static constexpr int kStageBytes = 2 * KS::kBytes;
   static constexpr int kSmemBytes = 2 * QT::kBytes + kStages * kStageBytes + 1024;
+  static constexpr int kBufs = 3;  // score buffers in TMEM
   // TMEM columns: S/dS and dP of buffer b, then dQ.
   __device__ static constexpr uint32_t col_s(int b) { return 128u * b; }
   __device__ static constexpr uint32_t col_dp(int b) { return 64u + 128u * b; }
-  static constexpr uint32_t kColDQ = 256;
+  static constexpr uint32_t kColDQ = 128 * kBufs;
+  static_assert(kColDQ + D <= 512, "TMEM columns");
 };
 
 template <int D, typename GradT>
@@ -425,8 +434,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __shared__ __align__(8) uint64_t q_full;
   __shared__ __align__(8) uint64_t st_full[C::kStages];
   __shared__ __align__(8) uint64_t st_empty[C::kStages];
-  __shared__ __align__(8) uint64_t s_full[2];
-  __shared__ __align__(8) uint64_t p_ready[2];
+  __shared__ __align__(8) uint64_t s_full[C::kBufs];
+  __shared__ __align__(8) uint64_t p_ready[C::kBufs];
   __shared__ __align__(8) uint64_t mma_done;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -454,7 +463,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&st_full[s], 1);
       mbar_init(&st_empty[s], 1);
     }
-    for (int t = 0; t < 2; ++t) {
+    for (int t = 0; t < C::kBufs; ++t) {
       mbar_init(&s_full[t], 1);
       mbar_init(&p_ready[t], 4);
     }
@@ -495,7 +504,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int l = max(0, s - C::kStages); l < s; ++l) mbar_drain(&st_full[l % C::kStages], (l / C::kStages) & 1);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {  // MMA issuer: whole warp, lane 0 issues
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);  // M=128 rows, N=64 keys
       constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, 0, 1);   // M=128 rows, N=D, B MN-major
       // Descriptors built once; each MMA adds a constant offset.
@@ -504,21 +513,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t st_kd = KS::kmajor_base(smem_addr(stages));
       const uint64_t st_mn = KS::mnmajor_base(smem_addr(stages));
       auto issue_scores = [&](int s) {
-        const int buf = s & 1;
+        const int buf = s % C::kBufs;
         const uint64_t k_kd = desc_advance(st_kd, (s % C::kStages) * C::kStageBytes);
         const uint64_t v_kd = desc_advance(k_kd, KS::kBytes);
+        // S and dP accumulate separately: alternate their K steps.
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + C::col_s(buf), desc_advance(q_kd, QT::kmajor_off(kk)), desc_advance(k_kd, KS::kmajor_off(kk)),
+        for (int kk = 0; kk < D / 16; ++kk) {
+          mma_ss_w(tmem + C::col_s(buf), desc_advance(q_kd, QT::kmajor_off(kk)), desc_advance(k_kd, KS::kmajor_off(kk)),
                  idesc_s, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + C::col_dp(buf), desc_advance(do_kd, QT::kmajor_off(kk)),
+          mma_ss_w(tmem + C::col_dp(buf), desc_advance(do_kd, QT::kmajor_off(kk)),
                  desc_advance(v_kd, KS::kmajor_off(kk)), idesc_s, kk > 0);
-        mma_commit(&s_full[buf]);
+        }
+        mma_commit_w(&s_full[buf]);
       };
       bool ok = mbar_wait(&q_full, 0, &abort_flag);
-      for (int s = 0; s < 2 && s < n_steps && ok; ++s) {
+      for (int s = 0; s < C::kBufs && s < n_steps && ok; ++s) {
         ok = mbar_wait(&st_full[s % C::kStages], (s / C::kStages) & 1, &abort_flag);
         if (ok) {
           tc_fence_after();
@@ -526,22 +535,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
       for (int s = 0; s < n_steps && ok; ++s) {
-        const int buf = s & 1;
-        if (!mbar_wait(&p_ready[buf], (s >> 1) & 1, &abort_flag)) break;
+        const int buf = s % C::kBufs;
+        if (!mbar_wait(&p_ready[buf], (s / C::kBufs) & 1, &abort_flag)) break;
         tc_fence_after();
         const uint64_t k_mn = desc_advance(st_mn, (s % C::kStages) * C::kStageBytes);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // 64 keys = 4 x K16
-          mma_ts(tmem + C::kColDQ, tmem + C::col_s(buf) + kk * 8, desc_advance(k_mn, KS::mnmajor_off(kk)), idesc_g,
+          mma_ts_w(tmem + C::kColDQ, tmem + C::col_s(buf) + kk * 8, desc_advance(k_mn, KS::mnmajor_off(kk)), idesc_g,
                  (s > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&st_empty[s % C::kStages]);
-        if (s + 2 < n_steps) {
-          if (!mbar_wait(&st_full[(s + 2) % C::kStages], ((s + 2) / C::kStages) & 1, &abort_flag)) break;
+        mma_commit_w(&st_empty[s % C::kStages]);
+        if (s + C::kBufs < n_steps) {  // the next scores into the buffer just read
+          const int s2 = s + C::kBufs;
+          if (!mbar_wait(&st_full[s2 % C::kStages], (s2 / C::kStages) & 1, &abort_flag)) break;
           tc_fence_after();
-          issue_scores(s + 2);
+          issue_scores(s2);
         }
       }
-      mma_commit(&mma_done);
+      mma_commit_w(&mma_done);
     }
   }
   } else {
@@ -561,16 +571,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint64_t ndd2 = f2_pack(ndd, ndd);
     bool ok = true;
     for (int s = grp; s < n_steps; s += 2) {
-      if (!mbar_wait(&s_full[grp], (s >> 1) & 1, &abort_flag)) {
+      const int buf = s % C::kBufs;
+      if (!mbar_wait(&s_full[buf], (s / C::kBufs) & 1, &abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
       uint32_t sr[64], dr[64];
-      tmem_ld32(lane_base + C::col_s(grp), *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(lane_base + C::col_s(grp) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld32(lane_base + C::col_dp(grp), *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
-      tmem_ld32(lane_base + C::col_dp(grp) + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+      tmem_ld32(lane_base + C::col_s(buf), *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(lane_base + C::col_s(buf) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(lane_base + C::col_dp(buf), *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+      tmem_ld32(lane_base + C::col_dp(buf) + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
       const int kbase = s * 64;
       int hi = p.N - kbase;                        // keys [0, hi) are < N
       if (p.causal) hi = min(hi, tok - kbase + 1);  // keys <= tok
@@ -605,11 +616,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         body(BoolC<false>{});
       else
         body(BoolC<true>{});
-      tmem_st32(lane_base + C::col_s(grp), dk);
+      tmem_st32(lane_base + C::col_s(buf), dk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_ready[grp]);
+      if (lane == 0) mbar_arrive(&p_ready[buf]);
     }
     if (ok) ok = mbar_wait(&mma_done, 0, &abort_flag);
     if (ok) {

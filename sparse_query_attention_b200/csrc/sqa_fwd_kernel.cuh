@@ -182,7 +182,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
   } else if (warp == 1) {
     // ======================= MMA issuer ===================================
-    if (lane == 0) {
+    // The whole warp runs this loop (warp-uniform values stay in uniform
+    // registers, which keeps each tcgen05.mma issue short); lane 0 issues.
+    {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t col_s[2] = {C::kColS0, C::kColS1};
@@ -199,7 +201,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int kk = 0; kk < D / 16; ++kk) {
           constexpr int kPerChunk = C::kRowElems / 16;
           const uint32_t off = (kk / kPerChunk) * C::kChunkBytes + (kk % kPerChunk) * 32;
-          mma_ss(tmem + col_s[t], desc_advance(a0, off), desc_advance(b0, off), idesc_s, kk > 0);
+          mma_ss_w(tmem + col_s[t], desc_advance(a0, off), desc_advance(b0, off), idesc_s, kk > 0);
         }
       };
       // Four 16-key MMAs over keys [16 k0, 16 k0 + 64).
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint64_t b0 = desc_advance(ring_mn, slot * C::kTileBytes);
 #pragma unroll
         for (int kk = k0; kk < k0 + 4; ++kk)
-          mma_ts(tmem + col_o[t], tmem + col_s[t] + kk * 8, desc_advance(b0, kk * 16 * C::kRowBytes), idesc_o,
+          mma_ts_w(tmem + col_o[t], tmem + col_s[t] + kk * 8, desc_advance(b0, kk * 16 * C::kRowBytes), idesc_o,
                  (acc || kk > k0) ? 1u : 0u);
       };
 
@@ -218,10 +220,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
-        mma_commit(&s_full[0]);
+        mma_commit_w(&s_full[0]);
         issue_s(1, 0);
-        mma_commit(&s_full[1]);
-        mma_commit(&slot_empty[0]);
+        mma_commit_w(&s_full[1]);
+        mma_commit_w(&slot_empty[0]);
       }
       for (int i = 0; i < n_steps && ok; ++i) {
         const int vpos = 2 * i + 1, kpos = 2 * i + 2;
@@ -237,10 +239,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (!mbar_wait(&p_ready[0][1], i & 1, &abort_flag)) break;
         tc_fence_after();
         issue_pv(0, vs, true, 4);
-        mma_commit(&o_done[0]);
+        mma_commit_w(&o_done[0]);
         if (more) {
           issue_s(0, ks);
-          mma_commit(&s_full[0]);
+          mma_commit_w(&s_full[0]);
         }
         // tile 1
         if (!mbar_wait(&p_ready[1][0], i & 1, &abort_flag)) break;
@@ -249,16 +251,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (!mbar_wait(&p_ready[1][1], i & 1, &abort_flag)) break;
         tc_fence_after();
         issue_pv(1, vs, true, 4);
-        mma_commit(&o_done[1]);
-        mma_commit(&slot_empty[vs]);
+        mma_commit_w(&o_done[1]);
+        mma_commit_w(&slot_empty[vs]);
         if (more) {
           issue_s(1, ks);
-          mma_commit(&s_full[1]);
-          mma_commit(&slot_empty[ks]);
+          mma_commit_w(&s_full[1]);
+          mma_commit_w(&slot_empty[ks]);
         }
       }
       (void)kslot;
-      mma_commit(&mma_done);
+      mma_commit_w(&mma_done);
     }
   }
   } else {

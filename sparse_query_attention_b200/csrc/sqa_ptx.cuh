@@ -185,6 +185,42 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                : "memory");
 }
 
+// Warp-wide forms: every lane of the warp executes the call with the same
+// operands (warp-uniform code, so they stay in uniform registers) and lane 0
+// alone issues the instruction.  The commit must come from the lane that
+// issued the MMAs, which lane 0 always is.
+__device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, l;\n\t.reg .u32 ln;\n\t"
+      "mov.u32 ln, %%laneid;\n\t"
+      "setp.eq.u32 l, ln, 0;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@l tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, l;\n\t.reg .u32 ln;\n\t"
+      "mov.u32 ln, %%laneid;\n\t"
+      "setp.eq.u32 l, ln, 0;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@l tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit_w(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred l;\n\t.reg .u32 ln;\n\t"
+      "mov.u32 ln, %%laneid;\n\t"
+      "setp.eq.u32 l, ln, 0;\n\t"
+      "@l tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(
+          smem_addr(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
