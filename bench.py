@@ -44,6 +44,30 @@ def attn_fwd_flops(B, N, H_q, d, causal):
     return 4 * B * H_q * P_c * d
 
 
+def rank_barrier(world):
+    """Barrier across the ranks of the default process group (no-op alone)."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def dist_max(value, world, device):
+    """Max of a float over all ranks (the job's time is its slowest rank's)."""
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_rate(world, units_per_rank_step, steps, max_ms):
+    """Whole-job rate: every rank processes its own problem each step, the job
+    takes as long as the slowest rank (max_ms over `steps` steps)."""
+    return world * units_per_rank_step * steps / (max_ms / 1e3)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -130,7 +154,7 @@ class ClockSampler:
 # ----------------------------------------------------------------------------
 # CPU baseline: the oracle as it stands, on a bounded sample of the workload.
 # ----------------------------------------------------------------------------
-def cpu_baseline(rows_per_head=128, seed=2):
+def cpu_baseline(rows_per_head=6144, seed=2):
     import numpy as np
     import torch
     from oracle import attention_forward
@@ -265,16 +289,11 @@ def run_sqa(args):
         sqa.sqa_attn_fwd(q, k, v, o, B, N, h_q, h_kv, d, w["causal"], scale, stream=stream)
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        rank_barrier(world)
         torch.cuda.synchronize(dev)
 
     def max_over_ranks(val):
-        if world == 1:
-            return val
-        t = torch.tensor([val], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return dist_max(val, world, dev)
 
     for _ in range(args.warmup):
         step(x["q"], x["k"], x["v"], out)
@@ -295,8 +314,8 @@ def run_sqa(args):
     per_launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = max_over_ranks(sum(per_launch_ms))
     ms_per_step = total_ms / args.steps
-    value = world * flops_step * args.steps / (total_ms / 1e3) / 1e12
-    tokens_per_s = world * B * N * args.steps / (total_ms / 1e3)
+    value = weak_scaling_rate(world, flops_step, args.steps, total_ms) / 1e12
+    tokens_per_s = weak_scaling_rate(world, B * N, args.steps, total_ms)
 
     # --- end to end through the C ABI with host buffers --------------------
     hq, hk, hv = (t.cpu().pin_memory() for t in (x["q"], x["k"], x["v"]))
@@ -319,7 +338,7 @@ def run_sqa(args):
     e1.record(stream)
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = world * flops_step * e2e_steps / (e2e_ms / 1e3) / 1e12
+    e2e_value = weak_scaling_rate(world, flops_step, e2e_steps, e2e_ms) / 1e12
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = ho.numel() * ho.element_size()
 

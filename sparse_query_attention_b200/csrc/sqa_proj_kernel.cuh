@@ -90,25 +90,25 @@ __global__ void __launch_bounds__(128, 1)
     // No copy may still be landing in shared memory when the CTA exits.
     for (int kb = issued > kProjStages ? issued - kProjStages : 0; kb < issued; ++kb)
       mbar_drain(&full_bar[kb % kProjStages], (kb / kProjStages) & 1);
-  } else if (warp == 1 && lane == 0) {
-    // MMA issuer
+  } else if (warp == 1) {
+    // MMA issuer: the whole warp runs the loop (operands stay warp-uniform),
+    // lane 0 issues.  Descriptors are built once and advanced by offsets.
     constexpr uint32_t idesc = idesc_bf16_f32(kProjBM, BN, 0, 0);
+    const uint64_t a_desc0 = smem_desc(smem_addr(a_tiles), 16, 1024, kSw128);
+    const uint64_t b_desc0 = smem_desc(smem_addr(b_tiles), 16, 1024, kSw128);
     for (int kb = 0; kb < num_kb; ++kb) {
       const int s = kb % kProjStages;
       const uint32_t ph = (kb / kProjStages) & 1;
       if (!mbar_wait(&full_bar[s], ph, &abort_flag)) break;
       tc_fence_after();
-      const uint32_t a0 = smem_addr(a_tiles + s * S::kABytes);
-      const uint32_t b0 = smem_addr(b_tiles + s * S::kBBytes);
+      const uint64_t ad = desc_advance(a_desc0, s * S::kABytes);
+      const uint64_t bd = desc_advance(b_desc0, s * S::kBBytes);
 #pragma unroll
-      for (int kk = 0; kk < kProjBK / 16; ++kk) {
-        const uint64_t ad = smem_desc(a0 + kk * 32, 16, 1024, kSw128);
-        const uint64_t bd = smem_desc(b0 + kk * 32, 16, 1024, kSw128);
-        mma_ss(tacc, ad, bd, idesc, (kb | kk) != 0);
-      }
-      mma_commit(&empty_bar[s]);
+      for (int kk = 0; kk < kProjBK / 16; ++kk)
+        mma_ss_w(tacc, desc_advance(ad, kk * 32), desc_advance(bd, kk * 32), idesc, (kb | kk) != 0);
+      mma_commit_w(&empty_bar[s]);
     }
-    mma_commit(&acc_bar);
+    mma_commit_w(&acc_bar);
   }
   __syncwarp();
 
