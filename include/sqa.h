@@ -155,6 +155,16 @@ sqa_status_t sqa_proj(const void* x, const void* w, const float* bias, void* y,
  */
 sqa_status_t sqa_device_status(void* stream);
 
+/*
+ * sqa_selftest_wait_timeout - exercises the bounded-wait failure path on the
+ * GPU without faulting anything: launches one warp that waits on a barrier
+ * nothing arrives on, gives up after timeout_ms (1..10000) and records
+ * SQA_ERR_TIMEOUT in the device status word, then returns normally.  A later
+ * sqa_device_status() reports (and clears) it; the context stays usable.
+ * Returns SQA_ERR_INVALID_ARG for an out-of-range timeout.
+ */
+sqa_status_t sqa_selftest_wait_timeout(int timeout_ms, void* stream);
+
 /* Static, human-readable name of a status code. */
 const char* sqa_status_string(sqa_status_t status);
 

@@ -38,6 +38,7 @@ SIGNATURES = {
                                  _I, _I, _I, _I, _I, _I, _F, _P]),
     "sqa_proj": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "sqa_device_status": (_I, [_P]),
+    "sqa_selftest_wait_timeout": (_I, [_I, _P]),
     "sqa_status_string": (ctypes.c_char_p, [_I]),
     "sqa_version": (ctypes.c_char_p, []),
 }
@@ -155,3 +156,7 @@ def sqa_proj(x, w, bias, y, y_dtype, M, K, Nout, stream=None) -> None:
 
 def sqa_device_status(stream=None) -> None:
     _check(library().sqa_device_status(_stream(stream)), "sqa_device_status")
+
+
+def sqa_selftest_wait_timeout(timeout_ms, stream=None) -> None:
+    _check(library().sqa_selftest_wait_timeout(int(timeout_ms), _stream(stream)), "sqa_selftest_wait_timeout")

@@ -425,6 +425,12 @@ sqa_status_t sqa_device_status(void* stream) {
   return SQA_OK;
 }
 
+sqa_status_t sqa_selftest_wait_timeout(int timeout_ms, void* stream) {
+  if (timeout_ms < 1 || timeout_ms > 10000) return SQA_ERR_INVALID_ARG;
+  sqa::selftest_wait_timeout_kernel<<<1, 32, 0, as_stream(stream)>>>(static_cast<uint64_t>(timeout_ms) * 1000000ull);
+  return launch_status();
+}
+
 const char* sqa_status_string(sqa_status_t status) {
   switch (status) {
     case SQA_OK: return "SQA_OK";

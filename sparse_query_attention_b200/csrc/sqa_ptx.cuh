@@ -66,7 +66,8 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 // kWaitLimitNs or as soon as *abort is non-zero; on giving up it records the
 // timeout, raises *abort so the other roles of the CTA wind down too, and
 // returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                              uint64_t limit_ns) {
   const uint32_t a = smem_addr(bar);
   if (mbar_test(a, parity)) return true;
   const uint64_t t0 = global_timer_ns();
@@ -75,12 +76,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     for (int i = 0; i < 32; ++i)
       if (mbar_test(a, parity)) return true;
     if (*abort) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       atomicOr(&g_status_word, kStatusTimeout);
       *abort = 1;
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return mbar_wait_for(bar, parity, abort, kWaitLimitNs);
+}
+
+// Self-test of the bounded wait: one warp waits on an mbarrier that nothing
+// ever arrives on; after limit_ns the wait gives up and records the timeout
+// in the status word, and the kernel returns normally.
+__global__ void selftest_wait_timeout_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t never;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&never, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  mbar_wait_for(&never, 0, &abort_flag, limit_ns);
 }
 
 // Teardown wait: bounded by time only (ignores *abort).  Used before a CTA

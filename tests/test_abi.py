@@ -105,6 +105,12 @@ def test_proj_rejects_invalid_arguments():
     assert lib.sqa_proj(FAKE, FAKE, None, FAKE, 0, 128, 64, 24, None) == sqa.SQA_ERR_UNSUPPORTED
 
 
+def test_selftest_rejects_out_of_range_timeout():
+    lib = sqa.library()
+    assert lib.sqa_selftest_wait_timeout(0, None) == sqa.SQA_ERR_INVALID_ARG
+    assert lib.sqa_selftest_wait_timeout(20000, None) == sqa.SQA_ERR_INVALID_ARG
+
+
 def test_binding_raises_on_error_status():
     with pytest.raises(sqa.SQAError) as e:
         sqa.sqa_attn_fwd(FAKE, FAKE, FAKE, FAKE, 1, 8, 4, 3, 32, True, 0.1, stream=0)
