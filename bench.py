@@ -211,6 +211,57 @@ def run_reference(args):
 TRAIN = {"B": 4, "N": 8192, "H_q": 8, "H_kv": 4, "d_head": 64, "causal": True}
 
 
+LAYER = {"B": 16, "N": 1024, "d_model": 256, "d_head": 16, "causal": True}
+LAYER_VARIANTS = {"MHA": (16, 16), "GQA": (16, 4), "SQA": (8, 4), "sSQA": (8, 8), "xSQA": (4, 4), "xSMQA": (4, 1)}
+
+
+def time_decoder_layer(sqa, torch, stream, flush, dev, reps=5):
+    """Forward of the small decoder attention layer (B=16, N=1024, d_model=256,
+    d_head=16, causal): Q/K/V projections at reduced width, the core, and the
+    output projection, per head-count variant (median of reps, L2 flushed)."""
+    from sqa_inputs import layer_inputs
+
+    c = LAYER
+    B, N, dm, dh = c["B"], c["N"], c["d_model"], c["d_head"]
+    M = B * N
+    P_c = N * (N + 1) // 2
+    out = {}
+    for name, (hq, hkv) in LAYER_VARIANTS.items():
+        x = layer_inputs(B, N, dm, hq, hkv, dh, seed=1, device=dev)
+        q = torch.empty((M, hq * dh), dtype=torch.bfloat16, device=dev)
+        k = torch.empty((M, hkv * dh), dtype=torch.bfloat16, device=dev)
+        v = torch.empty((M, hkv * dh), dtype=torch.bfloat16, device=dev)
+        o = torch.empty((M, hq * dh), dtype=torch.bfloat16, device=dev)
+        y = torch.empty((M, dm), dtype=torch.float32, device=dev)
+
+        def layer():
+            sqa.sqa_proj(x["x"], x["wq"], None, q, sqa.SQA_DT_BF16, M, dm, hq * dh, stream=stream)
+            sqa.sqa_proj(x["x"], x["wk"], None, k, sqa.SQA_DT_BF16, M, dm, hkv * dh, stream=stream)
+            sqa.sqa_proj(x["x"], x["wv"], None, v, sqa.SQA_DT_BF16, M, dm, hkv * dh, stream=stream)
+            sqa.sqa_attn_fwd_ex(q, k, v, o, sqa.SQA_DT_BF16, None, B, N, hq, hkv, dh, True, 1 / math.sqrt(dh),
+                                stream=stream)
+            sqa.sqa_proj(o, x["wo"], None, y, sqa.SQA_DT_F32, M, hq * dh, dm, stream=stream)
+
+        for _ in range(3):
+            layer()
+        times = []
+        for _ in range(reps):
+            flush.fill_(3)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            layer()
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        ms = statistics.median(times)
+        flops = 2 * M * dm * (hq + 2 * hkv) * dh + 2 * M * hq * dh * dm + 4 * B * hq * P_c * dh
+        out[name] = {"H_q": hq, "H_kv": hkv, "ms": ms, "tflops": flops / ms / 1e9, "tokens_per_s": M / (ms / 1e3)}
+    for name in out:
+        out[name]["speedup_vs_gqa"] = out["GQA"]["ms"] / out[name]["ms"]
+    sqa.sqa_device_status(stream)
+    return {"config": dict(c), "launches_per_layer": 5, "variants": out}
+
+
 def time_training_step(sqa, torch, stream, flush, dev, reps=5):
     """Causal SQA core forward + backward at B=4, N=8192, H_q=8, H_kv=4, d=64
     (bf16 inputs, fp32 gradients): median over reps, L2 flushed before each."""
@@ -367,6 +418,7 @@ def run_sqa(args):
         variants[name]["ideal_speedup"] = VARIANTS["MHA"][0] / variants[name]["H_q"]
     sqa.sqa_device_status(stream)
     training = time_training_step(sqa, torch, stream, flush, dev)
+    layer = time_decoder_layer(sqa, torch, stream, flush, dev)
 
     peak, peak_kind = load_peaks()
     achieved = flops_step / (statistics.mean(per_launch_ms) / 1e3) / 1e12
@@ -386,6 +438,7 @@ def run_sqa(args):
         "gpu_launches": args.steps,
         "variants": variants,
         "training_step": training,
+        "decoder_layer": layer,
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -82,6 +82,13 @@ def test_fwd_large_scores_and_custom_scale(sqa, causal):
     _check_fwd(sqa, 1, 640, 4, 4, 64, causal, seed=5, scale=1.0, mult=1.25)
 
 
+@pytest.mark.parametrize("H_q,H_kv,causal", [(6, 2, True), (12, 4, False), (6, 1, True), (24, 8, False)])
+def test_fwd_group_not_power_of_two(sqa, H_q, H_kv, causal):
+    """G = 3 or 6: the tile packs the largest power of two dividing G and a
+    KV head's query heads span several CTAs."""
+    _check_fwd(sqa, 2, 333, H_q, H_kv, 64, causal, seed=60 + H_q)
+
+
 def test_fwd_mha_mqa_extremes(sqa):
     _check_fwd(sqa, 1, 384, 16, 16, 64, True, seed=9)   # MHA
     _check_fwd(sqa, 1, 384, 16, 1, 64, False, seed=10)  # MQA-style single KV head

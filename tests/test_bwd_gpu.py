@@ -52,5 +52,12 @@ def test_bwd_shape_sweep(sqa, B, N, H_q, H_kv, d, causal):
     _check_bwd(sqa, B, N, H_q, H_kv, d, causal, seed=2000 + N)
 
 
+@pytest.mark.parametrize("H_q,H_kv,d,causal", [(6, 2, 64, True), (12, 4, 32, False), (6, 1, 128, True)])
+def test_bwd_group_not_power_of_two(sqa, H_q, H_kv, d, causal):
+    """G = 3 or 6: dK/dV sum over all G heads of the group; dQ tiles pack the
+    largest power of two dividing G."""
+    _check_bwd(sqa, 1, 300, H_q, H_kv, d, causal, seed=70 + H_q)
+
+
 def test_bwd_bf16_io(sqa):
     _check_bwd(sqa, 2, 384, 8, 4, 64, True, seed=21, o_dtype=torch.bfloat16, grad_dtype=torch.bfloat16)
