@@ -11,5 +11,7 @@ from .sqa_oracle import (  # noqa: F401
     attention_forward,
     attention_backward,
     projection,
+    projection_backward,
+    sqa_layer_backward,
     sqa_layer_forward,
 )

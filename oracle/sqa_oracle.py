@@ -165,3 +165,28 @@ def sqa_layer_forward(x, wq, wk, wv, wo, B: int, N: int, H_q: int, H_kv: int,
     o2 = o.reshape(B * N, H_q * d_head)
     y = projection(o2, wo)
     return {"q": q, "k": k, "v": v, "o": o2, "lse": lse, "y": y}
+
+
+def projection_backward(x, w, dy):
+    """Gradients of L = sum(y * dy) for y = x w^T: dx = dy w, dw = dy^T x."""
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    dy = np.asarray(dy, dtype=np.float64)
+    return dy @ w, dy.T @ x
+
+
+def sqa_layer_backward(x, wq, wk, wv, wo, dy, B: int, N: int, H_q: int, H_kv: int,
+                       d_head: int, causal: bool = True, scale=None):
+    """Gradient of the SQA layer above for L = sum(y * dy), all in fp64:
+    output projection, attention core (attention_backward), then the three
+    reduced-width input projections, whose input gradients add up in dx.
+    Returns dx [B*N, d_model], dwq, dwk, dwv, dwo (shapes of the weights)."""
+    if scale is None:
+        scale = 1.0 / np.sqrt(d_head)
+    fwd = sqa_layer_forward(x, wq, wk, wv, wo, B, N, H_q, H_kv, d_head, causal, scale)
+    do2, dwo = projection_backward(fwd["o"], wo, dy)
+    dq, dk, dv = attention_backward(fwd["q"], fwd["k"], fwd["v"], do2.reshape(B, N, H_q, d_head), causal, scale)
+    dxq, dwq = projection_backward(x, wq, dq.reshape(B * N, H_q * d_head))
+    dxk, dwk = projection_backward(x, wk, dk.reshape(B * N, H_kv * d_head))
+    dxv, dwv = projection_backward(x, wv, dv.reshape(B * N, H_kv * d_head))
+    return {"dx": dxq + dxk + dxv, "dwq": dwq, "dwk": dwk, "dwv": dwv, "dwo": dwo}

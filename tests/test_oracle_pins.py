@@ -21,7 +21,8 @@ import pytest
 import torch
 import torch.nn.functional as F
 
-from oracle import attention_backward, attention_forward, projection, sqa_layer_forward
+from oracle import (attention_backward, attention_forward, projection, projection_backward, sqa_layer_backward,
+                    sqa_layer_forward)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "closed_form_cases.json")
 
@@ -351,6 +352,46 @@ def test_layer_against_torch_composition():
     to = F.scaled_dot_product_attention(tq, tk, tv, is_causal=True, enable_gqa=True)
     ty = F.linear(to.transpose(1, 2).reshape(B * N, H_q * dh), torch.from_numpy(wo))
     np.testing.assert_allclose(out["y"], ty.numpy(), atol=1e-12)
+
+
+def test_projection_backward_brute_force():
+    """dx = dy w and dw = dy^T x against explicit sums (tiny)."""
+    rng = np.random.default_rng(23)
+    M, K, Nout = 4, 3, 5
+    x, w, dy = _rand((M, K), rng), _rand((Nout, K), rng), _rand((M, Nout), rng)
+    dx, dw = projection_backward(x, w, dy)
+    for m in range(M):
+        for k in range(K):
+            assert dx[m, k] == pytest.approx(math.fsum(dy[m, n] * w[n, k] for n in range(Nout)), abs=1e-13)
+    for n in range(Nout):
+        for k in range(K):
+            assert dw[n, k] == pytest.approx(math.fsum(dy[m, n] * x[m, k] for m in range(M)), abs=1e-13)
+
+
+@pytest.mark.parametrize("heads", [(4, 2), (4, 4), (4, 1)])
+def test_layer_backward_matches_autograd(heads):
+    """Every layer gradient equals torch autograd (fp64) through
+    linear -> SDPA (GQA) -> linear."""
+    H_q, H_kv = heads
+    rng = np.random.default_rng(29 + H_q + H_kv)
+    B, N, d_model, dh = 2, 13, 16, 8
+    x = _rand((B * N, d_model), rng)
+    wq = _rand((H_q * dh, d_model), rng, .2)
+    wk, wv = _rand((H_kv * dh, d_model), rng, .2), _rand((H_kv * dh, d_model), rng, .2)
+    wo = _rand((d_model, H_q * dh), rng, .2)
+    dy = _rand((B * N, d_model), rng)
+    g = sqa_layer_backward(x, wq, wk, wv, wo, dy, B, N, H_q, H_kv, dh, causal=True)
+    t = {n: torch.from_numpy(a.copy()).requires_grad_() for n, a in
+         (("x", x), ("wq", wq), ("wk", wk), ("wv", wv), ("wo", wo))}
+    tq = F.linear(t["x"], t["wq"]).view(B, N, H_q, dh).transpose(1, 2)
+    tk = F.linear(t["x"], t["wk"]).view(B, N, H_kv, dh).transpose(1, 2)
+    tv = F.linear(t["x"], t["wv"]).view(B, N, H_kv, dh).transpose(1, 2)
+    to = F.scaled_dot_product_attention(tq, tk, tv, is_causal=True, enable_gqa=H_q != H_kv)
+    ty = F.linear(to.transpose(1, 2).reshape(B * N, H_q * dh), t["wo"])
+    ty.backward(torch.from_numpy(dy))
+    np.testing.assert_allclose(g["dx"], t["x"].grad.numpy(), atol=1e-12)
+    for n in ("wq", "wk", "wv", "wo"):
+        np.testing.assert_allclose(g["d" + n], t[n].grad.numpy(), atol=1e-12)
 
 
 def test_rejects_bad_head_counts():
