@@ -148,6 +148,29 @@ sqa_status_t sqa_proj(const void* x, const void* w, const float* bias, void* y,
                       sqa_dtype_t y_dtype, int M, int K, int Nout, void* stream);
 
 /*
+ * sqa_gemm - the general projection contraction, used for the backward of
+ * the projections of an SQA layer (dX = dY W, dW = dY^T X) as well as the
+ * forward sqa_proj is a special case of:
+ *     C[M, N] (+)= sum_k A(m, k) B(n, k)  (+ bias[n])
+ * Operands are read as stored, no transpose through memory:
+ *   A(m, k) = a[m * K + k]  (SQA_K_CONTIGUOUS)  or  a[k * M + m]  (SQA_MN_CONTIGUOUS)
+ *   B(n, k) = b[n * K + k]  (SQA_K_CONTIGUOUS, nn.Linear weight layout)
+ *                        or  b[k * N + n]  (SQA_MN_CONTIGUOUS)
+ * a, b bf16; c row-major [M, N] in c_dtype; bias NULL or fp32 [N].
+ * accumulate != 0 adds into the existing C (fp32 C only).
+ * Requirements: M, N, K >= 1; K % 16 == 0; N % 16 == 0; M % 16 == 0 when A
+ * is MN-contiguous.  Examples (y = x W^T, x [M, K], W [N, K]):
+ *   forward  y  = sqa_gemm(x, K_CONTIGUOUS, W, K_CONTIGUOUS)            (M, N, K)
+ *   input    dx = sqa_gemm(dy, K_CONTIGUOUS, W, MN_CONTIGUOUS)          (M, K, N)
+ *   weight   dW = sqa_gemm(dy, MN_CONTIGUOUS, x, MN_CONTIGUOUS)         (N, K, M)
+ */
+typedef enum { SQA_K_CONTIGUOUS = 0, SQA_MN_CONTIGUOUS = 1 } sqa_layout_t;
+
+sqa_status_t sqa_gemm(const void* a, sqa_layout_t a_layout, const void* b, sqa_layout_t b_layout,
+                      const float* bias, void* c, sqa_dtype_t c_dtype, int accumulate,
+                      int M, int N, int K, void* stream);
+
+/*
  * sqa_device_status - synchronises `stream`, then returns SQA_ERR_TIMEOUT if
  * any kernel of this library on the current device gave up a bounded wait
  * since the last call (and clears the record), SQA_ERR_CUDA if the stream

@@ -26,6 +26,9 @@ SQA_ERR_TIMEOUT = 4
 SQA_DT_F32 = 0
 SQA_DT_BF16 = 1
 
+SQA_K_CONTIGUOUS = 0
+SQA_MN_CONTIGUOUS = 1
+
 # Every symbol include/sqa.h declares, with (restype, argtypes).
 _P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
@@ -37,6 +40,7 @@ SIGNATURES = {
     "sqa_attn_bwd_static": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I,
                                  _I, _I, _I, _I, _I, _I, _F, _P]),
     "sqa_proj": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "sqa_gemm": (_I, [_P, _I, _P, _I, _P, _P, _I, _I, _I, _I, _I, _P]),
     "sqa_device_status": (_I, [_P]),
     "sqa_selftest_wait_timeout": (_I, [_I, _P]),
     "sqa_status_string": (ctypes.c_char_p, [_I]),
@@ -152,6 +156,11 @@ def sqa_attn_bwd_static(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype
 def sqa_proj(x, w, bias, y, y_dtype, M, K, Nout, stream=None) -> None:
     _check(library().sqa_proj(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), int(y_dtype), M, K, Nout,
                          _stream(stream)), "sqa_proj")
+
+
+def sqa_gemm(a, a_layout, b, b_layout, bias, c, c_dtype, accumulate, M, N, K, stream=None) -> None:
+    _check(library().sqa_gemm(_ptr(a), int(a_layout), _ptr(b), int(b_layout), _ptr(bias), _ptr(c), int(c_dtype),
+                              int(bool(accumulate)), M, N, K, _stream(stream)), "sqa_gemm")
 
 
 def sqa_device_status(stream=None) -> None:

@@ -275,36 +275,70 @@ sqa_status_t launch_bwd_d(bool grad_bf16, const void* q, const void* k, const vo
 // ---------------------------------------------------------------------------
 // Projection GEMM
 // ---------------------------------------------------------------------------
-template <int BN, bool kBf16>
-sqa_status_t launch_proj_bn(const CUtensorMap& mx, const CUtensorMap& mw, const float* bias, void* y, int M, int K,
-                            int Nout, cudaStream_t st) {
-  auto kern = sqa::proj_gemm_kernel<BN, kBf16>;
+template <int BN, bool kBf16, bool kAMN, bool kBMN>
+sqa_status_t launch_gemm_bn(const CUtensorMap& ma, const CUtensorMap& mb, const float* bias, void* c, int M, int N,
+                            int K, int accumulate, cudaStream_t st) {
+  auto kern = sqa::proj_gemm_kernel<BN, kBf16, kAMN, kBMN>;
   constexpr int smem = sqa::ProjSmem<BN>::kDynamicBytes;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return SQA_ERR_CUDA;
-  dim3 grid((M + kProjBM - 1) / kProjBM, (Nout + BN - 1) / BN);
-  kern<<<grid, 128, smem, st>>>(mx, mw, bias, y, M, K, Nout);
+  dim3 grid((M + kProjBM - 1) / kProjBM, (N + BN - 1) / BN);
+  kern<<<grid, 128, smem, st>>>(ma, mb, bias, c, M, K, N, accumulate);
   return launch_status();
 }
 
-template <bool kBf16>
-sqa_status_t launch_proj(const CUtensorMap& mx, const void* w, const float* bias, void* y, int M, int K, int Nout,
-                         cudaStream_t st) {
-  // BN: the narrowest tile that covers Nout, at most 256.
-  int bn = 16;
-  while (bn < Nout && bn < 256) bn *= 2;
-  CUtensorMap mw;
-  const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(Nout)};
-  const uint64_t strides[1] = {static_cast<uint64_t>(K) * 2};
-  const uint32_t box[2] = {64, static_cast<uint32_t>(bn)};
-  if (!make_map_bf16(&mw, w, 2, dims, strides, box)) return SQA_ERR_CUDA;
+template <bool kBf16, bool kAMN, bool kBMN>
+sqa_status_t launch_gemm_layouts(const CUtensorMap& ma, const CUtensorMap& mb, int bn, const float* bias, void* c,
+                                 int M, int N, int K, int accumulate, cudaStream_t st) {
   switch (bn) {
-    case 16: return launch_proj_bn<16, kBf16>(mx, mw, bias, y, M, K, Nout, st);
-    case 32: return launch_proj_bn<32, kBf16>(mx, mw, bias, y, M, K, Nout, st);
-    case 64: return launch_proj_bn<64, kBf16>(mx, mw, bias, y, M, K, Nout, st);
-    case 128: return launch_proj_bn<128, kBf16>(mx, mw, bias, y, M, K, Nout, st);
-    default: return launch_proj_bn<256, kBf16>(mx, mw, bias, y, M, K, Nout, st);
+    case 16:
+      if constexpr (!kBMN) return launch_gemm_bn<16, kBf16, kAMN, kBMN>(ma, mb, bias, c, M, N, K, accumulate, st);
+      break;
+    case 32:
+      if constexpr (!kBMN) return launch_gemm_bn<32, kBf16, kAMN, kBMN>(ma, mb, bias, c, M, N, K, accumulate, st);
+      break;
+    case 64: return launch_gemm_bn<64, kBf16, kAMN, kBMN>(ma, mb, bias, c, M, N, K, accumulate, st);
+    case 128: return launch_gemm_bn<128, kBf16, kAMN, kBMN>(ma, mb, bias, c, M, N, K, accumulate, st);
+    default: return launch_gemm_bn<256, kBf16, kAMN, kBMN>(ma, mb, bias, c, M, N, K, accumulate, st);
   }
+  return SQA_ERR_UNSUPPORTED;
+}
+
+// C[M, N] (+)= sum_k A(m, k) B(n, k) (+ bias) with A, B K- or MN-contiguous.
+sqa_status_t gemm_impl(const void* a, bool a_mn, const void* b, bool b_mn, const float* bias, void* c,
+                       sqa_dtype_t c_dtype, int accumulate, int M, int N, int K, void* stream) {
+  if (!a || !b || !c) return SQA_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0) return SQA_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(b) || !aligned16(c) || (bias && !aligned16(bias))) return SQA_ERR_INVALID_ARG;
+  if (c_dtype != SQA_DT_F32 && c_dtype != SQA_DT_BF16) return SQA_ERR_INVALID_ARG;
+  if (accumulate && c_dtype != SQA_DT_F32) return SQA_ERR_INVALID_ARG;
+  if (K % 16 != 0 || N % 16 != 0 || (a_mn && M % 16 != 0)) return SQA_ERR_UNSUPPORTED;
+  // BN: the narrowest tile covering N, at most 256 (at least 64 when B is
+  // MN-contiguous: its tiles are loaded as 64-column boxes).
+  int bn = b_mn ? 64 : 16;
+  while (bn < N && bn < 256) bn *= 2;
+  CUtensorMap ma, mb;
+  const uint64_t a_dims[2] = {uint64_t(a_mn ? M : K), uint64_t(a_mn ? K : M)};
+  const uint64_t a_strides[1] = {uint64_t(a_mn ? M : K) * 2};
+  const uint32_t a_box[2] = {64, a_mn ? 64u : uint32_t(kProjBM)};
+  const uint64_t b_dims[2] = {uint64_t(b_mn ? N : K), uint64_t(b_mn ? K : N)};
+  const uint64_t b_strides[1] = {uint64_t(b_mn ? N : K) * 2};
+  const uint32_t b_box[2] = {64, b_mn ? 64u : uint32_t(bn)};
+  if (!make_map_bf16(&ma, a, 2, a_dims, a_strides, a_box) || !make_map_bf16(&mb, b, 2, b_dims, b_strides, b_box))
+    return SQA_ERR_CUDA;
+  cudaStream_t st = as_stream(stream);
+  const bool bf = c_dtype == SQA_DT_BF16;
+  if (!a_mn && !b_mn)
+    return bf ? launch_gemm_layouts<true, false, false>(ma, mb, bn, bias, c, M, N, K, accumulate, st)
+              : launch_gemm_layouts<false, false, false>(ma, mb, bn, bias, c, M, N, K, accumulate, st);
+  if (!a_mn && b_mn)
+    return bf ? launch_gemm_layouts<true, false, true>(ma, mb, bn, bias, c, M, N, K, accumulate, st)
+              : launch_gemm_layouts<false, false, true>(ma, mb, bn, bias, c, M, N, K, accumulate, st);
+  if (a_mn && b_mn)
+    return bf ? launch_gemm_layouts<true, true, true>(ma, mb, bn, bias, c, M, N, K, accumulate, st)
+              : launch_gemm_layouts<false, true, true>(ma, mb, bn, bias, c, M, N, K, accumulate, st);
+  return bf ? launch_gemm_layouts<true, true, false>(ma, mb, bn, bias, c, M, N, K, accumulate, st)
+            : launch_gemm_layouts<false, true, false>(ma, mb, bn, bias, c, M, N, K, accumulate, st);
 }
 
 }  // namespace
@@ -398,19 +432,16 @@ sqa_status_t sqa_attn_bwd_static(const void* q, const void* k, const void* v, co
 
 sqa_status_t sqa_proj(const void* x, const void* w, const float* bias, void* y, sqa_dtype_t y_dtype, int M, int K,
                       int Nout, void* stream) {
-  if (!x || !w || !y) return SQA_ERR_INVALID_ARG;
-  if (M <= 0 || K <= 0 || Nout <= 0) return SQA_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(w) || !aligned16(y) || (bias && !aligned16(bias))) return SQA_ERR_INVALID_ARG;
-  if (y_dtype != SQA_DT_F32 && y_dtype != SQA_DT_BF16) return SQA_ERR_INVALID_ARG;
-  if (K % 16 != 0 || Nout % 16 != 0) return SQA_ERR_UNSUPPORTED;
-  CUtensorMap mx;
-  const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
-  const uint64_t strides[1] = {static_cast<uint64_t>(K) * 2};
-  const uint32_t box[2] = {64, static_cast<uint32_t>(kProjBM)};
-  if (!make_map_bf16(&mx, x, 2, dims, strides, box)) return SQA_ERR_CUDA;
-  cudaStream_t st = as_stream(stream);
-  return y_dtype == SQA_DT_BF16 ? launch_proj<true>(mx, w, bias, y, M, K, Nout, st)
-                                : launch_proj<false>(mx, w, bias, y, M, K, Nout, st);
+  return gemm_impl(x, false, w, false, bias, y, y_dtype, 0, M, Nout, K, stream);
+}
+
+sqa_status_t sqa_gemm(const void* a, sqa_layout_t a_layout, const void* b, sqa_layout_t b_layout, const float* bias,
+                      void* c, sqa_dtype_t c_dtype, int accumulate, int M, int N, int K, void* stream) {
+  if ((a_layout != SQA_K_CONTIGUOUS && a_layout != SQA_MN_CONTIGUOUS) ||
+      (b_layout != SQA_K_CONTIGUOUS && b_layout != SQA_MN_CONTIGUOUS))
+    return SQA_ERR_INVALID_ARG;
+  return gemm_impl(a, a_layout == SQA_MN_CONTIGUOUS, b, b_layout == SQA_MN_CONTIGUOUS, bias, c, c_dtype,
+                   accumulate ? 1 : 0, M, N, K, stream);
 }
 
 sqa_status_t sqa_device_status(void* stream) {

@@ -1,17 +1,22 @@
-// sqa_proj_kernel.cuh - the reduced-width projection GEMM on the sm_100a
-// tensor cores:  Y[M, Nout] = X[M, K] * W[Nout, K]^T (+ bias).
+// sqa_proj_kernel.cuh - the projection GEMMs of an SQA layer on the sm_100a
+// tensor cores:  C[M, N] (+)= sum_k A(m, k) B(n, k) (+ bias[n]).
 //
 // In Sparse Query Attention the query projection produces only H_q * d_head
 // columns and the output projection consumes only H_q * d_head ("ReactiveAI/
 // xSMQAT-m" model card, note on model size); the key/value projections keep
-// H_kv * d_head.  All four are this one contraction.
+// H_kv * d_head.  The forward of all four is C = X W^T; their backward is
+// dX = dY W and dW = dY^T X.  The operands are therefore taken as stored,
+// either K-contiguous (A[m][k], B[n][k]: activations, nn.Linear weights) or
+// MN-contiguous (A[k][m], B[k][n]), and read with the matching shared-memory
+// operand layout, so no transpose ever goes through memory.
 //
 // Design: one CTA per 128 x BN output tile, four warps.
-//   warp 0 / one lane : TMA producer, 64-wide K slices of X and W into a
-//                       4-stage ring (128-byte swizzle, K-major).
-//   warp 1 / one lane : issues tcgen05.mma (M=128, N=BN, K=16) into a TMEM
-//                       accumulator, commits each stage back to the producer.
-//   all four warps    : epilogue, TMEM -> registers (+bias) -> global.
+//   warp 0 / one lane : TMA producer, 64-wide K slices of A and B into a
+//                       4-stage ring (128-byte swizzle).
+//   warp 1            : issues tcgen05.mma (M=128, N=BN, K=16) into a TMEM
+//                       accumulator from warp-uniform code (lane 0 issues),
+//                       commits each stage back to the producer.
+//   all four warps    : epilogue, TMEM -> registers (+C, +bias) -> global.
 #pragma once
 
 #include "sqa_ptx.cuh"
@@ -30,12 +35,17 @@ struct ProjSmem {
   static constexpr int kDynamicBytes = kTileBytes + 1024;  // + alignment slack
 };
 
-template <int BN, bool kOutBf16>
+// kAMN / kBMN: operand stored MN-contiguous (A[k][m] / B[k][n]) instead of
+// K-contiguous (A[m][k] / B[n][k]).  An MN-contiguous tile is loaded as
+// 64 (MN) x 64 (K) boxes, one 8 KB chunk per 64 rows of M or N.
+template <int BN, bool kOutBf16, bool kAMN, bool kBMN>
 __global__ void __launch_bounds__(128, 1)
-    proj_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                     const float* __restrict__ bias, void* __restrict__ y, int M, int K, int Nout) {
+    proj_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                     const float* __restrict__ bias, void* __restrict__ y, int M, int K, int Nout, int accumulate) {
+  static_assert(!kBMN || BN % 64 == 0, "MN-contiguous B needs BN in 64, 128, 256");
   using S = ProjSmem<BN>;
   constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
+  constexpr uint32_t kMnChunk = 64 * 128;  // one 64 x 64 MN-contiguous box
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kProjStages];
   __shared__ __align__(8) uint64_t empty_bar[kProjStages];
@@ -67,8 +77,8 @@ __global__ void __launch_bounds__(128, 1)
     tmem_relinquish();
   }
   if (warp == 1 && lane == 0) {
-    tma_prefetch_desc(&tm_x);
-    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
   }
   tc_fence_before();
   __syncthreads();
@@ -83,8 +93,20 @@ __global__ void __launch_bounds__(128, 1)
       const uint32_t ph = (kb / kProjStages) & 1;
       if (kb >= kProjStages && !mbar_wait(&empty_bar[s], ph ^ 1, &abort_flag)) break;
       mbar_arrive_expect_tx(&full_bar[s], S::kABytes + S::kBBytes);
-      tma_load_2d(&tm_x, &full_bar[s], a_tiles + s * S::kABytes, kb * kProjBK, m0);
-      tma_load_2d(&tm_w, &full_bar[s], b_tiles + s * S::kBBytes, kb * kProjBK, n0);
+      uint8_t* a_dst = a_tiles + s * S::kABytes;
+      uint8_t* b_dst = b_tiles + s * S::kBBytes;
+      if constexpr (kAMN) {
+        for (int c = 0; c < kProjBM / 64; ++c)
+          tma_load_2d(&tm_a, &full_bar[s], a_dst + c * kMnChunk, m0 + 64 * c, kb * kProjBK);
+      } else {
+        tma_load_2d(&tm_a, &full_bar[s], a_dst, kb * kProjBK, m0);
+      }
+      if constexpr (kBMN) {
+        for (int c = 0; c < BN / 64; ++c)
+          tma_load_2d(&tm_b, &full_bar[s], b_dst + c * kMnChunk, n0 + 64 * c, kb * kProjBK);
+      } else {
+        tma_load_2d(&tm_b, &full_bar[s], b_dst, kb * kProjBK, n0);
+      }
       ++issued;
     }
     // No copy may still be landing in shared memory when the CTA exits.
@@ -92,10 +114,17 @@ __global__ void __launch_bounds__(128, 1)
       mbar_drain(&full_bar[kb % kProjStages], (kb / kProjStages) & 1);
   } else if (warp == 1) {
     // MMA issuer: the whole warp runs the loop (operands stay warp-uniform),
-    // lane 0 issues.  Descriptors are built once and advanced by offsets.
-    constexpr uint32_t idesc = idesc_bf16_f32(kProjBM, BN, 0, 0);
-    const uint64_t a_desc0 = smem_desc(smem_addr(a_tiles), 16, 1024, kSw128);
-    const uint64_t b_desc0 = smem_desc(smem_addr(b_tiles), 16, 1024, kSw128);
+    // lane 0 issues.  Descriptors are built once and advanced by offsets:
+    // a K-contiguous operand steps 32 bytes along its 128-byte rows per
+    // 16-wide K step; an MN-contiguous one steps 16 rows of 128 bytes, with
+    // its 64-wide MN chunks kMnChunk bytes apart.
+    constexpr uint32_t idesc = idesc_bf16_f32(kProjBM, BN, kAMN ? 1 : 0, kBMN ? 1 : 0);
+    const uint64_t a_desc0 = kAMN ? smem_desc(smem_addr(a_tiles), kMnChunk, 1024, kSw128)
+                                  : smem_desc(smem_addr(a_tiles), 16, 1024, kSw128);
+    const uint64_t b_desc0 = kBMN ? smem_desc(smem_addr(b_tiles), kMnChunk, 1024, kSw128)
+                                  : smem_desc(smem_addr(b_tiles), 16, 1024, kSw128);
+    constexpr uint32_t kAStep = kAMN ? 16 * 128 : 32;
+    constexpr uint32_t kBStep = kBMN ? 16 * 128 : 32;
     for (int kb = 0; kb < num_kb; ++kb) {
       const int s = kb % kProjStages;
       const uint32_t ph = (kb / kProjStages) & 1;
@@ -105,7 +134,7 @@ __global__ void __launch_bounds__(128, 1)
       const uint64_t bd = desc_advance(b_desc0, s * S::kBBytes);
 #pragma unroll
       for (int kk = 0; kk < kProjBK / 16; ++kk)
-        mma_ss_w(tacc, desc_advance(ad, kk * 32), desc_advance(bd, kk * 32), idesc, (kb | kk) != 0);
+        mma_ss_w(tacc, desc_advance(ad, kk * kAStep), desc_advance(bd, kk * kBStep), idesc, (kb | kk) != 0);
       mma_commit_w(&empty_bar[s]);
     }
     mma_commit_w(&acc_bar);
@@ -137,13 +166,23 @@ __global__ void __launch_bounds__(128, 1)
         } else {
           float4* dst = reinterpret_cast<float4*>(static_cast<float*>(y) + static_cast<size_t>(row) * Nout + n);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          for (int i = 0; i < 4; ++i) {
+            float4 w = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            if (accumulate) {
+              const float4 old = dst[i];
+              w.x += old.x;
+              w.y += old.y;
+              w.z += old.z;
+              w.w += old.w;
+            }
+            dst[i] = w;
+          }
         }
       }
     }
   }
-  // The MMA thread always commits acc_bar, so this returns once every MMA
-  // it issued has finished, also after an abort.
+  // The MMA warp always commits acc_bar, so this returns once every MMA it
+  // issued has finished, also after an abort.
   if (!ok && threadIdx.x == 0) mbar_drain(&acc_bar, 0);
   tc_fence_before();
   __syncthreads();
