@@ -234,32 +234,69 @@ def time_decoder_layer(sqa, torch, stream, flush, dev, reps=5):
         o = torch.empty((M, hq * dh), dtype=torch.bfloat16, device=dev)
         y = torch.empty((M, dm), dtype=torch.float32, device=dev)
 
-        def layer():
-            sqa.sqa_proj(x["x"], x["wq"], None, q, sqa.SQA_DT_BF16, M, dm, hq * dh, stream=stream)
-            sqa.sqa_proj(x["x"], x["wk"], None, k, sqa.SQA_DT_BF16, M, dm, hkv * dh, stream=stream)
-            sqa.sqa_proj(x["x"], x["wv"], None, v, sqa.SQA_DT_BF16, M, dm, hkv * dh, stream=stream)
-            sqa.sqa_attn_fwd_ex(q, k, v, o, sqa.SQA_DT_BF16, None, B, N, hq, hkv, dh, True, 1 / math.sqrt(dh),
-                                stream=stream)
-            sqa.sqa_proj(o, x["wo"], None, y, sqa.SQA_DT_F32, M, hq * dh, dm, stream=stream)
+        lse = torch.empty((B, hq, N), dtype=torch.float32, device=dev)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(11)
+        dy = torch.randn((M, dm), generator=gen, device=dev).to(torch.bfloat16)
+        do = torch.empty_like(o)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        dx = torch.empty((M, dm), dtype=torch.float32, device=dev)
+        dws = {n: torch.empty((w * dh, dm), dtype=torch.float32, device=dev)
+               for n, w in (("wq", hq), ("wk", hkv), ("wv", hkv))}
+        dwo = torch.empty((dm, hq * dh), dtype=torch.float32, device=dev)
+        wsb = sqa.sqa_attn_bwd_workspace_size(B, N, hq, hkv, dh)
+        ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+        KC, MN, BF, F32 = sqa.SQA_K_CONTIGUOUS, sqa.SQA_MN_CONTIGUOUS, sqa.SQA_DT_BF16, sqa.SQA_DT_F32
+        sc = 1 / math.sqrt(dh)
 
-        for _ in range(3):
+        def layer():
+            sqa.sqa_proj(x["x"], x["wq"], None, q, BF, M, dm, hq * dh, stream=stream)
+            sqa.sqa_proj(x["x"], x["wk"], None, k, BF, M, dm, hkv * dh, stream=stream)
+            sqa.sqa_proj(x["x"], x["wv"], None, v, BF, M, dm, hkv * dh, stream=stream)
+            sqa.sqa_attn_fwd_ex(q, k, v, o, BF, lse, B, N, hq, hkv, dh, True, sc, stream=stream)
+            sqa.sqa_proj(o, x["wo"], None, y, F32, M, hq * dh, dm, stream=stream)
+
+        def layer_backward():
+            sqa.sqa_gemm(dy, KC, x["wo"], MN, None, do, BF, False, M, hq * dh, dm, stream=stream)
+            sqa.sqa_gemm(dy, MN, o, MN, None, dwo, F32, False, dm, hq * dh, M, stream=stream)
+            sqa.sqa_attn_bwd(q, k, v, o, BF, do, lse, dq, dk, dv, BF, B, N, hq, hkv, dh, True, sc, ws, wsb,
+                             stream=stream)
+            for i, (n, g_, w) in enumerate((("wq", dq, hq), ("wk", dk, hkv), ("wv", dv, hkv))):
+                sqa.sqa_gemm(g_, MN, x["x"], MN, None, dws[n], F32, False, w * dh, dm, M, stream=stream)
+                sqa.sqa_gemm(g_, KC, x[n], MN, None, dx, F32, i > 0, M, dm, w * dh, stream=stream)
+
+        def timed(fn):
+            for _ in range(3):
+                fn()
+            times = []
+            for _ in range(reps):
+                flush.fill_(3)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                b.synchronize()
+                times.append(a.elapsed_time(b))
+            return statistics.median(times)
+
+        def step():
             layer()
-        times = []
-        for _ in range(reps):
-            flush.fill_(3)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            layer()
-            b.record(stream)
-            b.synchronize()
-            times.append(a.elapsed_time(b))
-        ms = statistics.median(times)
-        flops = 2 * M * dm * (hq + 2 * hkv) * dh + 2 * M * hq * dh * dm + 4 * B * hq * P_c * dh
-        out[name] = {"H_q": hq, "H_kv": hkv, "ms": ms, "tflops": flops / ms / 1e9, "tokens_per_s": M / (ms / 1e3)}
+            layer_backward()
+
+        ms = timed(layer)
+        ms_train = timed(step)
+        proj_f = 2 * M * dm * (hq + 2 * hkv) * dh + 2 * M * hq * dh * dm
+        attn_f = 4 * B * hq * P_c * dh
+        flops = proj_f + attn_f
+        train_flops = 3 * proj_f + 3 * attn_f  # backward: 2x projections, 2x core (algorithmic)
+        out[name] = {"H_q": hq, "H_kv": hkv, "ms": ms, "tflops": flops / ms / 1e9, "tokens_per_s": M / (ms / 1e3),
+                     "train_ms": ms_train, "train_tflops": train_flops / ms_train / 1e9,
+                     "train_tokens_per_s": M / (ms_train / 1e3)}
     for name in out:
         out[name]["speedup_vs_gqa"] = out["GQA"]["ms"] / out[name]["ms"]
+        out[name]["train_speedup_vs_gqa"] = out["GQA"]["train_ms"] / out[name]["train_ms"]
     sqa.sqa_device_status(stream)
-    return {"config": dict(c), "launches_per_layer": 5, "variants": out}
+    return {"config": dict(c), "launches_forward": 5, "launches_training_step": 15, "variants": out}
 
 
 def time_training_step(sqa, torch, stream, flush, dev, reps=5):
