@@ -211,6 +211,45 @@ def run_reference(args):
 TRAIN = {"B": 4, "N": 8192, "H_q": 8, "H_kv": 4, "d_head": 64, "causal": True}
 
 
+LONG = {"B": 1, "d_head": 128, "causal": False, "N": (131072, 200000)}
+LONG_VARIANTS = {"MHA": (16, 16), "SQA": (8, 4), "xSQA": (4, 4)}
+
+
+def time_long_sequences(sqa, torch, stream, dev, reps=3):
+    """Non-causal core forward at N = 131072 and 200000 (B=1, d=128) for MHA,
+    SQA and xSQA on the same kernel: the long-sequence end of the 32k-200k
+    range.  Inputs are larger than L2, so no flush is needed."""
+    from sqa_inputs import attention_inputs
+
+    c = LONG
+    d = c["d_head"]
+    res = {}
+    for N in c["N"]:
+        per = {}
+        for name, (hq, hkv) in LONG_VARIANTS.items():
+            x = attention_inputs(1, N, hq, hkv, d, seed=3, device=dev)
+            o = torch.empty((1, N, hq * d), dtype=torch.float32, device=dev)
+            sqa.sqa_attn_fwd(x["q"], x["k"], x["v"], o, 1, N, hq, hkv, d, False, 1 / math.sqrt(d), stream=stream)
+            times = []
+            for _ in range(reps):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                sqa.sqa_attn_fwd(x["q"], x["k"], x["v"], o, 1, N, hq, hkv, d, False, 1 / math.sqrt(d),
+                                 stream=stream)
+                b.record(stream)
+                b.synchronize()
+                times.append(a.elapsed_time(b))
+            ms = statistics.median(times)
+            per[name] = {"H_q": hq, "H_kv": hkv, "ms": ms,
+                         "tflops": attn_fwd_flops(1, N, hq, d, False) / ms / 1e9, "tokens_per_s": N / (ms / 1e3)}
+            del x, o
+        for name in per:
+            per[name]["speedup_vs_mha"] = per["MHA"]["ms"] / per[name]["ms"]
+        res[str(N)] = per
+    sqa.sqa_device_status(stream)
+    return {"config": {"B": 1, "d_head": d, "causal": False}, "by_N": res}
+
+
 LAYER = {"B": 16, "N": 1024, "d_model": 256, "d_head": 16, "causal": True}
 LAYER_VARIANTS = {"MHA": (16, 16), "GQA": (16, 4), "SQA": (8, 4), "sSQA": (8, 8), "xSQA": (4, 4), "xSMQA": (4, 1)}
 
@@ -456,6 +495,7 @@ def run_sqa(args):
     sqa.sqa_device_status(stream)
     training = time_training_step(sqa, torch, stream, flush, dev)
     layer = time_decoder_layer(sqa, torch, stream, flush, dev)
+    long_seq = time_long_sequences(sqa, torch, stream, dev)
 
     peak, peak_kind = load_peaks()
     achieved = flops_step / (statistics.mean(per_launch_ms) / 1e3) / 1e12
@@ -476,6 +516,7 @@ def run_sqa(args):
         "variants": variants,
         "training_step": training,
         "decoder_layer": layer,
+        "long_sequences": long_seq,
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
