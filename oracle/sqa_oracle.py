@@ -48,6 +48,14 @@ def _check_heads(H_q: int, H_kv: int) -> int:
     return H_q // H_kv
 
 
+def _check_lengths(N_q: int, N_kv: int, causal: bool) -> None:
+    # Cross / memory attention (queries and keys of different lengths) is
+    # taken without a mask: "query t sees keys 0..t" has no meaning when the
+    # keys are not the same sequence.
+    if causal and N_q != N_kv:
+        raise ValueError("causal attention needs as many keys as queries")
+
+
 def _scores(q_rows, k_head, t_rows, causal, scale):
     """s[r, u] = scale * <q_r, k_u>, with u > t_r set to -inf when causal.
 
@@ -67,7 +75,9 @@ def _scores(q_rows, k_head, t_rows, causal, scale):
 def attention_forward(q, k, v, causal: bool, scale: float, rows=None):
     """Sparse Query Attention output and log-sum-exp.
 
-    q: [B, N, H_q, d]; k, v: [B, N, H_kv, d] (float64 arrays).
+    q: [B, N, H_q, d]; k, v: [B, N_kv, H_kv, d] (float64 arrays; N_kv = N
+    for self-attention, any length for cross / memory attention, which is
+    never causal).
     rows: optional 1-D array of query token indices; all rows when None.
     Returns o [B, R, H_q, d] and lse [B, H_q, R] (R = number of rows), with
         o[b,t,h]   = sum_u softmax_u(s_tu) v[b,u,j],  j = h // G
@@ -79,6 +89,7 @@ def attention_forward(q, k, v, causal: bool, scale: float, rows=None):
     B, N, H_q, d = q.shape
     H_kv = k.shape[2]
     G = _check_heads(H_q, H_kv)
+    _check_lengths(N, k.shape[1], causal)
     t_all = np.arange(N) if rows is None else np.asarray(rows, dtype=np.int64)
     R = t_all.shape[0]
     o = np.empty((B, R, H_q, d), dtype=np.float64)
@@ -116,6 +127,7 @@ def attention_backward(q, k, v, do, causal: bool, scale: float):
     B, N, H_q, d = q.shape
     H_kv = k.shape[2]
     G = _check_heads(H_q, H_kv)
+    _check_lengths(N, k.shape[1], causal)
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)

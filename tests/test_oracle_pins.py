@@ -394,6 +394,53 @@ def test_layer_backward_matches_autograd(heads):
         np.testing.assert_allclose(g["d" + n], t[n].grad.numpy(), atol=1e-12)
 
 
+@pytest.mark.parametrize("N_q,N_kv,heads", [(7, 19, (4, 2)), (33, 5, (4, 4)), (16, 64, (8, 1))])
+def test_cross_attention_matches_sdpa_and_autograd(N_q, N_kv, heads):
+    """Queries and keys of different lengths (memory attention): output and
+    all three gradients equal torch SDPA / autograd in fp64."""
+    H_q, H_kv = heads
+    rng = np.random.default_rng(N_q * 7 + N_kv)
+    B, d = 2, 8
+    q, k, v = _rand((B, N_q, H_q, d), rng), _rand((B, N_kv, H_kv, d), rng), _rand((B, N_kv, H_kv, d), rng)
+    do = _rand((B, N_q, H_q, d), rng)
+    scale = 1 / math.sqrt(d)
+    o, lse = attention_forward(q, k, v, False, scale)
+    tq, tk, tv = (torch.from_numpy(a.copy()).permute(0, 2, 1, 3).requires_grad_() for a in (q, k, v))
+    to = F.scaled_dot_product_attention(tq, tk, tv, scale=scale, enable_gqa=H_q != H_kv)
+    np.testing.assert_allclose(o, to.detach().permute(0, 2, 1, 3).numpy(), atol=1e-12)
+    ob, lseb = brute_attention_cross(q, k, v, scale)
+    np.testing.assert_allclose(lse, lseb, atol=1e-12)
+    to.backward(torch.from_numpy(do).permute(0, 2, 1, 3))
+    dq, dk, dv = attention_backward(q, k, v, do, False, scale)
+    np.testing.assert_allclose(dq, tq.grad.permute(0, 2, 1, 3).numpy(), atol=1e-12)
+    np.testing.assert_allclose(dk, tk.grad.permute(0, 2, 1, 3).numpy(), atol=1e-12)
+    np.testing.assert_allclose(dv, tv.grad.permute(0, 2, 1, 3).numpy(), atol=1e-12)
+
+
+def brute_attention_cross(q, k, v, scale):
+    """Non-causal brute force for different query / key lengths (fsum)."""
+    B, N_q, H_q, d = q.shape
+    N_kv, H_kv = k.shape[1], k.shape[2]
+    G = H_q // H_kv
+    o = np.zeros(q.shape)
+    lse = np.zeros((B, H_q, N_q))
+    for b in range(B):
+        for h in range(H_q):
+            for t in range(N_q):
+                e = [math.exp(scale * math.fsum(q[b, t, h, c] * k[b, u, h // G, c] for c in range(d)))
+                     for u in range(N_kv)]
+                z = math.fsum(e)
+                for c in range(d):
+                    o[b, t, h, c] = math.fsum(e[u] * v[b, u, h // G, c] for u in range(N_kv)) / z
+                lse[b, h, t] = math.log(z)
+    return o, lse
+
+
+def test_causal_cross_attention_is_rejected():
+    with pytest.raises(ValueError):
+        attention_forward(np.zeros((1, 3, 1, 2)), np.zeros((1, 5, 1, 2)), np.zeros((1, 5, 1, 2)), True, 1.0)
+
+
 def test_rejects_bad_head_counts():
     q = np.zeros((1, 2, 3, 4))
     k = np.zeros((1, 2, 2, 4))
