@@ -106,6 +106,39 @@ sqa_status_t sqa_attn_bwd(const void* q, const void* k, const void* v,
                           void* stream);
 
 /*
+ * sqa_attn_fwd_cross - cross / memory attention: N_q query tokens attend,
+ * without a mask, to N_kv key/value tokens of another sequence (a memory
+ * state, an encoder's output).  "ReactiveAI/GQA-Ref-Micro" model card,
+ * closing outlook: the Reactive Transformer's memory attention, designed with
+ * shared key/value heads, is to take SQA variants as well; "Sparse Query
+ * Attention ...", "Built on by" (Reactive Transformer).
+ * Layouts: q, out [B, N_q, H_q, d_head]; k, v [B, N_kv, H_kv, d_head] bf16;
+ *   lse [B, H_q, N_q] fp32 or NULL.
+ * Otherwise as sqa_attn_fwd_ex with causal = 0: N_q, N_kv >= 1, any pair
+ * (N_kv may be shorter or longer than N_q).  sqa_attn_fwd_ex(..., N, ...)
+ * equals sqa_attn_fwd_cross(..., N_q = N, N_kv = N, ...) non-causal.
+ */
+sqa_status_t sqa_attn_fwd_cross(const void* q, const void* k, const void* v, void* out,
+                                sqa_dtype_t out_dtype, float* lse,
+                                int B, int N_q, int N_kv, int H_q, int H_kv, int d_head,
+                                float scale, void* stream);
+
+/*
+ * sqa_attn_bwd_cross - gradient of sqa_attn_fwd_cross.  Arguments as
+ * sqa_attn_bwd with causal = 0 and the two lengths apart: q, out, dout, dq
+ * [B, N_q, H_q, d]; k, v, dk, dv [B, N_kv, H_kv, d]; lse [B, H_q, N_q].
+ * The workspace is sqa_attn_bwd_workspace_size(B, N_q, H_q, H_kv, d_head)
+ * bytes (it holds per-query-row values only).
+ */
+sqa_status_t sqa_attn_bwd_cross(const void* q, const void* k, const void* v,
+                                const void* out, sqa_dtype_t o_dtype,
+                                const void* dout, const float* lse,
+                                void* dq, void* dk, void* dv, sqa_dtype_t grad_dtype,
+                                int B, int N_q, int N_kv, int H_q, int H_kv, int d_head,
+                                float scale, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/*
  * sqa_attn_bwd_static - sqa_attn_bwd without a caller-supplied workspace.
  * (Library plumbing; the paper has no counterpart.)
  *

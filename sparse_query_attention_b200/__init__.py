@@ -34,9 +34,12 @@ _P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
     "sqa_attn_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "sqa_attn_fwd_ex": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "sqa_attn_fwd_cross": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "sqa_attn_bwd_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "sqa_attn_bwd": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I,
                           _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
+    "sqa_attn_bwd_cross": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I,
+                                _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "sqa_attn_bwd_static": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I,
                                  _I, _I, _I, _I, _I, _I, _F, _P]),
     "sqa_proj": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
@@ -129,6 +132,14 @@ def sqa_attn_fwd_ex(q, k, v, out, out_dtype, lse, B, N, H_q, H_kv, d_head, causa
                                 _stream(stream)), "sqa_attn_fwd_ex")
 
 
+def sqa_attn_fwd_cross(q, k, v, out, out_dtype, lse, B, N_q, N_kv, H_q, H_kv, d_head, scale,
+                       stream=None) -> None:
+    """Cross / memory attention: N_q queries, N_kv keys, no mask."""
+    _check(library().sqa_attn_fwd_cross(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(out_dtype), _ptr(lse),
+                                        B, N_q, N_kv, H_q, H_kv, d_head, float(scale),
+                                        _stream(stream)), "sqa_attn_fwd_cross")
+
+
 def sqa_attn_bwd_workspace_size(B, N, H_q, H_kv, d_head) -> int:
     return int(library().sqa_attn_bwd_workspace_size(B, N, H_q, H_kv, d_head))
 
@@ -140,6 +151,16 @@ def sqa_attn_bwd(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B, N,
                              B, N, H_q, H_kv, d_head, int(bool(causal)), float(scale),
                              _ptr(workspace), int(workspace_bytes), _stream(stream)),
            "sqa_attn_bwd")
+
+
+def sqa_attn_bwd_cross(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B, N_q, N_kv, H_q,
+                       H_kv, d_head, scale, workspace, workspace_bytes, stream=None) -> None:
+    """Gradient of sqa_attn_fwd_cross; workspace sized for N_q query rows."""
+    _check(library().sqa_attn_bwd_cross(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(o_dtype), _ptr(dout),
+                                        _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), int(grad_dtype),
+                                        B, N_q, N_kv, H_q, H_kv, d_head, float(scale),
+                                        _ptr(workspace), int(workspace_bytes), _stream(stream)),
+           "sqa_attn_bwd_cross")
 
 
 def sqa_attn_bwd_static(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B, N, H_q, H_kv,

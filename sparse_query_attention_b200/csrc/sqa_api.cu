@@ -74,6 +74,15 @@ sqa_status_t check_attn_args(const void* q, const void* k, const void* v, int B,
   return SQA_OK;
 }
 
+// Key/value length: any positive length without a mask (cross / memory
+// attention); a causal mask needs as many keys as queries.
+sqa_status_t check_kv_length(int B, int N, int Nkv, int H_kv, int causal) {
+  if (Nkv <= 0) return SQA_ERR_INVALID_ARG;
+  if (causal && Nkv != N) return SQA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * Nkv * H_kv > (1ll << 31) - 1) return SQA_ERR_UNSUPPORTED;
+  return SQA_OK;
+}
+
 // ---------------------------------------------------------------------------
 // Attention forward
 // ---------------------------------------------------------------------------
@@ -91,7 +100,7 @@ int head_pack(int G) {
 
 template <int D>
 sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* out, int out_bf16, float* lse, int B,
-                           int N, int H_q, int H_kv, int causal, float scale, cudaStream_t st) {
+                           int N, int Nkv, int H_q, int H_kv, int causal, float scale, cudaStream_t st) {
   using C = sqa::FwdCfg<D>;
   const int G = H_q / H_kv;
   const int g = head_pack(G);
@@ -107,8 +116,8 @@ sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* ou
     if (!make_map_bf16(&mq, q, 4, dims, strides, box, swz)) return SQA_ERR_CUDA;
   }
   {
-    const uint64_t dims[4] = {uint64_t(D), uint64_t(H_kv), uint64_t(N), uint64_t(B)};
-    const uint64_t strides[3] = {uint64_t(D) * 2, uint64_t(H_kv) * D * 2, uint64_t(N) * H_kv * D * 2};
+    const uint64_t dims[4] = {uint64_t(D), uint64_t(H_kv), uint64_t(Nkv), uint64_t(B)};
+    const uint64_t strides[3] = {uint64_t(D) * 2, uint64_t(H_kv) * D * 2, uint64_t(Nkv) * H_kv * D * 2};
     const uint32_t box[4] = {uint32_t(C::kRowElems), 1, 128, 1};
     if (!make_map_bf16(&mk, k, 4, dims, strides, box, swz)) return SQA_ERR_CUDA;
     if (!make_map_bf16(&mv, v, 4, dims, strides, box, swz)) return SQA_ERR_CUDA;
@@ -118,6 +127,7 @@ sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* ou
   p.lse = lse;
   p.B = B;
   p.N = N;
+  p.Nkv = Nkv;
   p.H_q = H_q;
   p.H_kv = H_kv;
   p.G = G;
@@ -139,18 +149,20 @@ sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* ou
 }
 
 sqa_status_t attn_fwd_impl(const void* q, const void* k, const void* v, void* out, sqa_dtype_t out_dtype, float* lse,
-                           int B, int N, int H_q, int H_kv, int d, int causal, float scale, void* stream) {
+                           int B, int N, int Nkv, int H_q, int H_kv, int d, int causal, float scale, void* stream) {
   sqa_status_t s = check_attn_args(q, k, v, B, N, H_q, H_kv, d, scale);
+  if (s != SQA_OK) return s;
+  s = check_kv_length(B, N, Nkv, H_kv, causal);
   if (s != SQA_OK) return s;
   if (!out || !aligned16(out) || (lse && !aligned16(lse))) return SQA_ERR_INVALID_ARG;
   if (out_dtype != SQA_DT_F32 && out_dtype != SQA_DT_BF16) return SQA_ERR_INVALID_ARG;
   const int ob = out_dtype == SQA_DT_BF16;
   cudaStream_t st = as_stream(stream);
   switch (d) {
-    case 16: return launch_fwd_tc<16>(q, k, v, out, ob, lse, B, N, H_q, H_kv, causal, scale, st);
-    case 32: return launch_fwd_tc<32>(q, k, v, out, ob, lse, B, N, H_q, H_kv, causal, scale, st);
-    case 64: return launch_fwd_tc<64>(q, k, v, out, ob, lse, B, N, H_q, H_kv, causal, scale, st);
-    default: return launch_fwd_tc<128>(q, k, v, out, ob, lse, B, N, H_q, H_kv, causal, scale, st);
+    case 16: return launch_fwd_tc<16>(q, k, v, out, ob, lse, B, N, Nkv, H_q, H_kv, causal, scale, st);
+    case 32: return launch_fwd_tc<32>(q, k, v, out, ob, lse, B, N, Nkv, H_q, H_kv, causal, scale, st);
+    case 64: return launch_fwd_tc<64>(q, k, v, out, ob, lse, B, N, Nkv, H_q, H_kv, causal, scale, st);
+    default: return launch_fwd_tc<128>(q, k, v, out, ob, lse, B, N, Nkv, H_q, H_kv, causal, scale, st);
   }
 }
 
@@ -192,8 +204,8 @@ bool make_map_bnhd(CUtensorMap* map, const void* base, int B, int N, int H, uint
 
 template <int D, typename GradT>
 sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const void* o, int o_bf16, const void* dout,
-                           const float* lse, void* dq, void* dk, void* dv, int B, int N, int H_q, int H_kv,
-                           int causal, float scale, void* workspace, cudaStream_t st) {
+                           const float* lse, void* dq, void* dk, void* dv, int B, int N, int Nkv, int H_q,
+                           int H_kv, int causal, float scale, void* workspace, cudaStream_t st) {
   const int n_pad = bwd_n_pad(N);
   float* dsum = static_cast<float*>(workspace);
   float* lse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + bwd_half_bytes(B, N, H_q));
@@ -211,6 +223,7 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
   p.lse2 = lse2;
   p.B = B;
   p.N = N;
+  p.Nkv = Nkv;
   p.H_q = H_q;
   p.H_kv = H_kv;
   p.G = G;
@@ -226,10 +239,10 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
   if (gy > 65535 || B > 65535) return SQA_ERR_UNSUPPORTED;
 
   CUtensorMap m_k128, m_v128, m_q64, m_do64, m_l2, m_ds, m_qp, m_dop, m_k64, m_v64;
-  if (!make_map_bnhd<D>(&m_k128, k, B, N, H_kv, 1, 128) || !make_map_bnhd<D>(&m_v128, v, B, N, H_kv, 1, 128) ||
+  if (!make_map_bnhd<D>(&m_k128, k, B, Nkv, H_kv, 1, 128) || !make_map_bnhd<D>(&m_v128, v, B, Nkv, H_kv, 1, 128) ||
       !make_map_bnhd<D>(&m_q64, q, B, N, H_q, 1, 64) || !make_map_bnhd<D>(&m_do64, dout, B, N, H_q, 1, 64) ||
       !make_map_bnhd<D>(&m_qp, q, B, N, H_q, g, T) || !make_map_bnhd<D>(&m_dop, dout, B, N, H_q, g, T) ||
-      !make_map_bnhd<D>(&m_k64, k, B, N, H_kv, 1, 64) || !make_map_bnhd<D>(&m_v64, v, B, N, H_kv, 1, 64) ||
+      !make_map_bnhd<D>(&m_k64, k, B, Nkv, H_kv, 1, 64) || !make_map_bnhd<D>(&m_v64, v, B, Nkv, H_kv, 1, 64) ||
       !make_map_f32_2d(&m_l2, lse2, n_pad, uint64_t(B) * H_q, 64) ||
       !make_map_f32_2d(&m_ds, dsum, n_pad, uint64_t(B) * H_q, 64))
     return SQA_ERR_CUDA;
@@ -246,7 +259,7 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
     constexpr int smem = sqa::DkdvCfg<D>::kSmemBytes;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return SQA_ERR_CUDA;
-    dim3 grid((N + 127) / 128, H_kv, B);
+    dim3 grid((Nkv + 127) / 128, H_kv, B);
     kern<<<grid, sqa::kBwdThreads, smem, st>>>(m_k128, m_v128, m_q64, m_do64, m_l2, m_ds, p);
     if (cudaGetLastError() != cudaSuccess) return SQA_ERR_CUDA;
   }
@@ -264,12 +277,47 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
 
 template <int D>
 sqa_status_t launch_bwd_d(bool grad_bf16, const void* q, const void* k, const void* v, const void* o, int o_bf16,
-                          const void* dout, const float* lse, void* dq, void* dk, void* dv, int B, int N, int H_q,
-                          int H_kv, int causal, float scale, void* ws, cudaStream_t st) {
+                          const void* dout, const float* lse, void* dq, void* dk, void* dv, int B, int N, int Nkv,
+                          int H_q, int H_kv, int causal, float scale, void* ws, cudaStream_t st) {
   if (grad_bf16)
-    return launch_bwd_tc<D, __nv_bfloat16>(q, k, v, o, o_bf16, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal,
+    return launch_bwd_tc<D, __nv_bfloat16>(q, k, v, o, o_bf16, dout, lse, dq, dk, dv, B, N, Nkv, H_q, H_kv, causal,
                                            scale, ws, st);
-  return launch_bwd_tc<D, float>(q, k, v, o, o_bf16, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, ws, st);
+  return launch_bwd_tc<D, float>(q, k, v, o, o_bf16, dout, lse, dq, dk, dv, B, N, Nkv, H_q, H_kv, causal, scale, ws,
+                                 st);
+}
+
+sqa_status_t attn_bwd_impl(const void* q, const void* k, const void* v, const void* out, sqa_dtype_t o_dtype,
+                           const void* dout, const float* lse, void* dq, void* dk, void* dv, sqa_dtype_t grad_dtype,
+                           int B, int N, int Nkv, int H_q, int H_kv, int d_head, int causal, float scale,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  sqa_status_t s = check_attn_args(q, k, v, B, N, H_q, H_kv, d_head, scale);
+  if (s != SQA_OK) return s;
+  s = check_kv_length(B, N, Nkv, H_kv, causal);
+  if (s != SQA_OK) return s;
+  if (!out || !dout || !lse || !dq || !dk || !dv || !workspace) return SQA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(dout) || !aligned16(lse) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv) || !aligned16(workspace))
+    return SQA_ERR_INVALID_ARG;
+  if ((o_dtype != SQA_DT_F32 && o_dtype != SQA_DT_BF16) || (grad_dtype != SQA_DT_F32 && grad_dtype != SQA_DT_BF16))
+    return SQA_ERR_INVALID_ARG;
+  if (workspace_bytes < bwd_workspace_bytes(B, N, H_q)) return SQA_ERR_INVALID_ARG;
+  const bool gb = grad_dtype == SQA_DT_BF16;
+  const int ob = o_dtype == SQA_DT_BF16;
+  cudaStream_t st = as_stream(stream);
+  switch (d_head) {
+    case 16:
+      return launch_bwd_d<16>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, Nkv, H_q, H_kv, causal, scale,
+                              workspace, st);
+    case 32:
+      return launch_bwd_d<32>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, Nkv, H_q, H_kv, causal, scale,
+                              workspace, st);
+    case 64:
+      return launch_bwd_d<64>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, Nkv, H_q, H_kv, causal, scale,
+                              workspace, st);
+    default:
+      return launch_bwd_d<128>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, Nkv, H_q, H_kv, causal, scale,
+                               workspace, st);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -347,13 +395,19 @@ extern "C" {
 
 sqa_status_t sqa_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int N, int H_q, int H_kv,
                           int d_head, int causal, float scale, void* stream) {
-  return attn_fwd_impl(q, k, v, out, SQA_DT_F32, nullptr, B, N, H_q, H_kv, d_head, causal, scale, stream);
+  return attn_fwd_impl(q, k, v, out, SQA_DT_F32, nullptr, B, N, N, H_q, H_kv, d_head, causal, scale, stream);
 }
 
 sqa_status_t sqa_attn_fwd_ex(const void* q, const void* k, const void* v, void* out, sqa_dtype_t out_dtype,
                              float* lse, int B, int N, int H_q, int H_kv, int d_head, int causal, float scale,
                              void* stream) {
-  return attn_fwd_impl(q, k, v, out, out_dtype, lse, B, N, H_q, H_kv, d_head, causal, scale, stream);
+  return attn_fwd_impl(q, k, v, out, out_dtype, lse, B, N, N, H_q, H_kv, d_head, causal, scale, stream);
+}
+
+sqa_status_t sqa_attn_fwd_cross(const void* q, const void* k, const void* v, void* out, sqa_dtype_t out_dtype,
+                                float* lse, int B, int N_q, int N_kv, int H_q, int H_kv, int d_head, float scale,
+                                void* stream) {
+  return attn_fwd_impl(q, k, v, out, out_dtype, lse, B, N_q, N_kv, H_q, H_kv, d_head, 0, scale, stream);
 }
 
 size_t sqa_attn_bwd_workspace_size(int B, int N, int H_q, int H_kv, int d_head) {
@@ -365,24 +419,16 @@ sqa_status_t sqa_attn_bwd(const void* q, const void* k, const void* v, const voi
                           const void* dout, const float* lse, void* dq, void* dk, void* dv, sqa_dtype_t grad_dtype,
                           int B, int N, int H_q, int H_kv, int d_head, int causal, float scale, void* workspace,
                           size_t workspace_bytes, void* stream) {
-  sqa_status_t s = check_attn_args(q, k, v, B, N, H_q, H_kv, d_head, scale);
-  if (s != SQA_OK) return s;
-  if (!out || !dout || !lse || !dq || !dk || !dv || !workspace) return SQA_ERR_INVALID_ARG;
-  if (!aligned16(out) || !aligned16(dout) || !aligned16(lse) || !aligned16(dq) || !aligned16(dk) ||
-      !aligned16(dv) || !aligned16(workspace))
-    return SQA_ERR_INVALID_ARG;
-  if ((o_dtype != SQA_DT_F32 && o_dtype != SQA_DT_BF16) || (grad_dtype != SQA_DT_F32 && grad_dtype != SQA_DT_BF16))
-    return SQA_ERR_INVALID_ARG;
-  if (workspace_bytes < bwd_workspace_bytes(B, N, H_q)) return SQA_ERR_INVALID_ARG;
-  const bool gb = grad_dtype == SQA_DT_BF16;
-  const int ob = o_dtype == SQA_DT_BF16;
-  cudaStream_t st = as_stream(stream);
-  switch (d_head) {
-    case 16: return launch_bwd_d<16>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, workspace, st);
-    case 32: return launch_bwd_d<32>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, workspace, st);
-    case 64: return launch_bwd_d<64>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, workspace, st);
-    default: return launch_bwd_d<128>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, H_q, H_kv, causal, scale, workspace, st);
-  }
+  return attn_bwd_impl(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B, N, N, H_q, H_kv, d_head, causal,
+                       scale, workspace, workspace_bytes, stream);
+}
+
+sqa_status_t sqa_attn_bwd_cross(const void* q, const void* k, const void* v, const void* out, sqa_dtype_t o_dtype,
+                                const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                                sqa_dtype_t grad_dtype, int B, int N_q, int N_kv, int H_q, int H_kv, int d_head,
+                                float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  return attn_bwd_impl(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B, N_q, N_kv, H_q, H_kv, d_head, 0,
+                       scale, workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"

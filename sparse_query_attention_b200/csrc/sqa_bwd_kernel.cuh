@@ -116,7 +116,8 @@ struct BwdParams {
   void* dv;
   const float* dsum;  // [B, H_q, n_pad]
   const float* lse2;  // [B, H_q, n_pad]
-  int B, N, H_q, H_kv, G, n_pad;
+  int B, N, H_q, H_kv, G, n_pad;  // N: query tokens, n_pad: N rounded up to 128
+  int Nkv;                        // key/value tokens (N for self-attention)
   int g, log2g, n_sub, n_tblk;  // packing of the dQ kernel
   int causal;
   float scale;
@@ -376,11 +377,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (ok) ok = mbar_wait(&mma_done, 0, &abort_flag);
     if (ok) {
       tc_fence_after();
-      const bool valid = u < p.N;
+      const bool valid = u < p.Nkv;
       const uint32_t col = grp == 0 ? C::kColDV : C::kColDK;
       const float mult = grp == 0 ? 1.f : p.scale;
       GradT* dst = static_cast<GradT*>(grp == 0 ? p.dv : p.dk) +
-                   ((static_cast<size_t>(b) * p.N + (valid ? u : 0)) * p.H_kv + j) * D;
+                   ((static_cast<size_t>(b) * p.Nkv + (valid ? u : 0)) * p.H_kv + j) * D;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 16) {
         uint32_t rr[16];
@@ -455,7 +456,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int h0 = j * p.G + sub * p.g;
   const int t0 = tblk * T;
   const int last_tok = min(t0 + T, p.N) - 1;
-  const int n_steps = p.causal ? (last_tok / 64 + 1) : (p.N + 63) / 64;  // 64-key sub-tiles
+  const int n_steps = p.causal ? (last_tok / 64 + 1) : (p.Nkv + 63) / 64;  // 64-key sub-tiles
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
@@ -583,7 +584,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tmem_ld32(lane_base + C::col_dp(buf), *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
       tmem_ld32(lane_base + C::col_dp(buf) + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
       const int kbase = s * 64;
-      int hi = p.N - kbase;                        // keys [0, hi) are < N
+      int hi = p.Nkv - kbase;                      // keys [0, hi) exist
       if (p.causal) hi = min(hi, tok - kbase + 1);  // keys <= tok
       const bool full = __all_sync(0xffffffffu, hi >= 64);
       tmem_wait_ld();

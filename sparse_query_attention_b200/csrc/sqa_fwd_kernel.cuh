@@ -56,7 +56,8 @@ struct FwdCfg {
 struct FwdParams {
   void* out;       // [B, N, H_q, D], fp32 or bf16
   float* lse;      // [B, H_q, N] or null
-  int B, N, H_q, H_kv, G, g, log2g;
+  int B, N, H_q, H_kv, G, g, log2g;  // N: query tokens
+  int Nkv;         // key/value tokens (N for self-attention; causal needs Nkv == N)
   int n_sub;       // G / g head sub-groups per KV head
   int n_tblk;      // token blocks of 2 * (128 / g) tokens
   int causal;
@@ -103,7 +104,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int b = blockIdx.z;
   const int h0 = j * p.G + sub * p.g;
   const int t0 = tblk * 2 * T;  // tile 0 tokens [t0, t0+T), tile 1 [t0+T, t0+2T)
-  const int n_kv_all = (p.N + 127) / 128;
+  const int n_kv_all = (p.Nkv + 127) / 128;
   int n_kv[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
@@ -301,10 +302,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // taken on them and the scale is folded into the exponent's FFMA.
       // Masked tiles are scaled first and get -inf where masked.
       const int key0 = i * 128;
-      const bool need_mask = (key0 + 128 > p.N) || (p.causal && key0 + 127 > tile_tok_min) || i >= n_kv[t];
+      const bool need_mask = (key0 + 128 > p.Nkv) || (p.causal && key0 + 127 > tile_tok_min) || i >= n_kv[t];
       float mult = sl2;  // exponent argument = s * mult - m
       if (need_mask) {
-        int lim = p.N - key0;                                   // keys [0, lim) are < N
+        int lim = p.Nkv - key0;                                 // keys [0, lim) exist
         if (p.causal) lim = min(lim, tok - key0 + 1);           // keys <= tok
         if (i >= n_kv[t]) lim = 0;
 #pragma unroll

@@ -47,6 +47,22 @@ def attention_inputs(B: int, N: int, H_q: int, H_kv: int, d_head: int, seed: int
     return out
 
 
+def cross_attention_inputs(B: int, N_q: int, N_kv: int, H_q: int, H_kv: int, d_head: int, seed: int,
+                           with_dout: bool = False, device="cpu") -> dict:
+    """Cross / memory attention: Q (and dO) [B,N_q,H_q,d], K and V
+    [B,N_kv,H_kv,d], bf16, drawn in the same order as attention_inputs."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    out = {
+        "q": _draw(gen, (B, N_q, H_q, d_head), 1.0, device),
+        "k": _draw(gen, (B, N_kv, H_kv, d_head), 1.0, device),
+        "v": _draw(gen, (B, N_kv, H_kv, d_head), 1.0, device),
+    }
+    if with_dout:
+        out["do"] = _draw(gen, (B, N_q, H_q, d_head), 1.0, device)
+    return out
+
+
 def layer_inputs(B: int, N: int, d_model: int, H_q: int, H_kv: int, d_head: int,
                  seed: int, device="cpu") -> dict:
     """x [B*N, d_model]; Wq [H_q*d, d_model]; Wk, Wv [H_kv*d, d_model];

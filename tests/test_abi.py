@@ -24,7 +24,7 @@ def _declared_symbols():
 def test_header_declares_expected_entry_points():
     names = _declared_symbols()
     for n in ("sqa_attn_fwd", "sqa_attn_fwd_ex", "sqa_attn_bwd", "sqa_attn_bwd_workspace_size",
-              "sqa_proj", "sqa_device_status", "sqa_status_string", "sqa_version"):
+              "sqa_attn_fwd_cross", "sqa_attn_bwd_cross", "sqa_proj", "sqa_device_status", "sqa_status_string", "sqa_version"):
         assert n in names
 
 
@@ -93,6 +93,19 @@ def test_bwd_rejects_invalid_arguments():
                dict(od=5), dict(gd=2), dict(H_kv=3), dict(dq=FAKE + 2)):
         assert call(**kw) == sqa.SQA_ERR_INVALID_ARG, kw
     assert call(d=80) == sqa.SQA_ERR_UNSUPPORTED
+
+
+def test_cross_rejects_invalid_lengths():
+    lib = sqa.library()
+    for n_q, n_kv in ((0, 8), (8, 0), (8, -1)):
+        assert lib.sqa_attn_fwd_cross(FAKE, FAKE, FAKE, FAKE, 0, None, 1, n_q, n_kv, 4, 2, 32, 0.1,
+                                      None) == sqa.SQA_ERR_INVALID_ARG
+    ws = sqa.sqa_attn_bwd_workspace_size(1, 8, 4, 2, 32)
+    assert lib.sqa_attn_bwd_cross(FAKE, FAKE, FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1, 8, 0, 4, 2, 32,
+                                  0.1, FAKE, ws, None) == sqa.SQA_ERR_INVALID_ARG
+    # The workspace holds per-query-row values: sized for N_q, not N_kv.
+    assert lib.sqa_attn_bwd_cross(FAKE, FAKE, FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1, 4096, 8, 4, 2, 32,
+                                  0.1, FAKE, ws, None) == sqa.SQA_ERR_INVALID_ARG
 
 
 def test_proj_rejects_invalid_arguments():
