@@ -255,9 +255,12 @@ LAYER_VARIANTS = {"MHA": (16, 16), "GQA": (16, 4), "SQA": (8, 4), "sSQA": (8, 8)
 
 
 def time_decoder_layer(sqa, torch, stream, flush, dev, reps=5):
-    """Forward of the small decoder attention layer (B=16, N=1024, d_model=256,
-    d_head=16, causal): Q/K/V projections at reduced width, the core, and the
-    output projection, per head-count variant (median of reps, L2 flushed)."""
+    """Forward and training step of the small decoder attention layer (B=16,
+    N=1024, d_model=256, d_head=16, causal), per head-count variant (median of
+    reps, L2 flushed).  The input projection is fused: one GEMM with the
+    concatenated weight [Wq; Wk; Wv] writes a packed QKV buffer that the
+    attention reads in place; the backward writes packed dQKV, so dX and
+    d[Wq; Wk; Wv] are one GEMM each.  Forward 3 launches, training step 10."""
     from sqa_inputs import layer_inputs
 
     c = LAYER
@@ -267,9 +270,9 @@ def time_decoder_layer(sqa, torch, stream, flush, dev, reps=5):
     out = {}
     for name, (hq, hkv) in LAYER_VARIANTS.items():
         x = layer_inputs(B, N, dm, hq, hkv, dh, seed=1, device=dev)
-        q = torch.empty((M, hq * dh), dtype=torch.bfloat16, device=dev)
-        k = torch.empty((M, hkv * dh), dtype=torch.bfloat16, device=dev)
-        v = torch.empty((M, hkv * dh), dtype=torch.bfloat16, device=dev)
+        W = (hq + 2 * hkv) * dh
+        w_qkv = torch.cat([x["wq"], x["wk"], x["wv"]], dim=0).contiguous()
+        qkv = torch.empty((M, W), dtype=torch.bfloat16, device=dev)
         o = torch.empty((M, hq * dh), dtype=torch.bfloat16, device=dev)
         y = torch.empty((M, dm), dtype=torch.float32, device=dev)
 
@@ -278,10 +281,9 @@ def time_decoder_layer(sqa, torch, stream, flush, dev, reps=5):
         gen.manual_seed(11)
         dy = torch.randn((M, dm), generator=gen, device=dev).to(torch.bfloat16)
         do = torch.empty_like(o)
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        dqkv = torch.empty_like(qkv)
         dx = torch.empty((M, dm), dtype=torch.float32, device=dev)
-        dws = {n: torch.empty((w * dh, dm), dtype=torch.float32, device=dev)
-               for n, w in (("wq", hq), ("wk", hkv), ("wv", hkv))}
+        dw_qkv = torch.empty((W, dm), dtype=torch.float32, device=dev)
         dwo = torch.empty((dm, hq * dh), dtype=torch.float32, device=dev)
         wsb = sqa.sqa_attn_bwd_workspace_size(B, N, hq, hkv, dh)
         ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
@@ -289,20 +291,17 @@ def time_decoder_layer(sqa, torch, stream, flush, dev, reps=5):
         sc = 1 / math.sqrt(dh)
 
         def layer():
-            sqa.sqa_proj(x["x"], x["wq"], None, q, BF, M, dm, hq * dh, stream=stream)
-            sqa.sqa_proj(x["x"], x["wk"], None, k, BF, M, dm, hkv * dh, stream=stream)
-            sqa.sqa_proj(x["x"], x["wv"], None, v, BF, M, dm, hkv * dh, stream=stream)
-            sqa.sqa_attn_fwd_ex(q, k, v, o, BF, lse, B, N, hq, hkv, dh, True, sc, stream=stream)
+            sqa.sqa_proj(x["x"], w_qkv, None, qkv, BF, M, dm, W, stream=stream)
+            sqa.sqa_attn_fwd_packed(qkv, o, BF, lse, B, N, hq, hkv, dh, True, sc, stream=stream)
             sqa.sqa_proj(o, x["wo"], None, y, F32, M, hq * dh, dm, stream=stream)
 
         def layer_backward():
             sqa.sqa_gemm(dy, KC, x["wo"], MN, None, do, BF, False, M, hq * dh, dm, stream=stream)
             sqa.sqa_gemm(dy, MN, o, MN, None, dwo, F32, False, dm, hq * dh, M, stream=stream)
-            sqa.sqa_attn_bwd(q, k, v, o, BF, do, lse, dq, dk, dv, BF, B, N, hq, hkv, dh, True, sc, ws, wsb,
-                             stream=stream)
-            for i, (n, g_, w) in enumerate((("wq", dq, hq), ("wk", dk, hkv), ("wv", dv, hkv))):
-                sqa.sqa_gemm(g_, MN, x["x"], MN, None, dws[n], F32, False, w * dh, dm, M, stream=stream)
-                sqa.sqa_gemm(g_, KC, x[n], MN, None, dx, F32, i > 0, M, dm, w * dh, stream=stream)
+            sqa.sqa_attn_bwd_packed(qkv, o, BF, do, lse, dqkv, BF, B, N, hq, hkv, dh, True, sc, ws, wsb,
+                                    stream=stream)
+            sqa.sqa_gemm(dqkv, KC, w_qkv, MN, None, dx, F32, False, M, dm, W, stream=stream)
+            sqa.sqa_gemm(dqkv, MN, x["x"], MN, None, dw_qkv, F32, False, W, dm, M, stream=stream)
 
         def timed(fn):
             for _ in range(3):
@@ -335,7 +334,7 @@ def time_decoder_layer(sqa, torch, stream, flush, dev, reps=5):
         out[name]["speedup_vs_gqa"] = out["GQA"]["ms"] / out[name]["ms"]
         out[name]["train_speedup_vs_gqa"] = out["GQA"]["train_ms"] / out[name]["train_ms"]
     sqa.sqa_device_status(stream)
-    return {"config": dict(c), "launches_forward": 5, "launches_training_step": 15, "variants": out}
+    return {"config": dict(c), "launches_forward": 3, "launches_training_step": 10, "fused_qkv": True, "variants": out}
 
 
 def time_training_step(sqa, torch, stream, flush, dev, reps=5):

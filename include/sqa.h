@@ -139,6 +139,37 @@ sqa_status_t sqa_attn_bwd_cross(const void* q, const void* k, const void* v,
                                 void* stream);
 
 /*
+ * sqa_attn_fwd_packed - the forward on a packed QKV buffer, the output of one
+ * fused input projection with the concatenated weight [Wq; Wk; Wv]
+ * ((H_q + 2 H_kv) * d_head rows): qkv [B, N, H_q + 2 H_kv, d_head] bf16,
+ * holding per token the H_q query heads, then the H_kv key heads, then the
+ * H_kv value heads.  SQA narrows exactly this projection (query and output
+ * projections of width H_q * d_head: "ReactiveAI/xSMQAT-m" model card, note
+ * on model size), so one GEMM produces all three operands.
+ * out [B, N, H_q, d_head] (out_dtype) and lse [B, H_q, N] (or NULL) are
+ * dense, as in sqa_attn_fwd_ex; every other argument and rule as there.
+ * The result equals sqa_attn_fwd_ex on the three heads' slices copied out.
+ */
+sqa_status_t sqa_attn_fwd_packed(const void* qkv, void* out, sqa_dtype_t out_dtype, float* lse,
+                                 int B, int N, int H_q, int H_kv, int d_head, int causal,
+                                 float scale, void* stream);
+
+/*
+ * sqa_attn_bwd_packed - gradient of sqa_attn_fwd_packed: dqkv
+ * [B, N, H_q + 2 H_kv, d_head] in grad_dtype, laid out as qkv (dQ heads,
+ * then dK, then dV), so the input projection's backward is one GEMM for dX
+ * and one for the concatenated weight gradient.  out, dout [B, N, H_q, d]
+ * and lse [B, H_q, N] are dense; workspace as sqa_attn_bwd.  Every entry of
+ * dqkv is overwritten.
+ */
+sqa_status_t sqa_attn_bwd_packed(const void* qkv, const void* out, sqa_dtype_t o_dtype,
+                                 const void* dout, const float* lse,
+                                 void* dqkv, sqa_dtype_t grad_dtype,
+                                 int B, int N, int H_q, int H_kv, int d_head, int causal,
+                                 float scale, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
+/*
  * sqa_attn_bwd_static - sqa_attn_bwd without a caller-supplied workspace.
  * (Library plumbing; the paper has no counterpart.)
  *

@@ -35,11 +35,14 @@ SIGNATURES = {
     "sqa_attn_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "sqa_attn_fwd_ex": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "sqa_attn_fwd_cross": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "sqa_attn_fwd_packed": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "sqa_attn_bwd_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "sqa_attn_bwd": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I,
                           _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "sqa_attn_bwd_cross": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I,
                                 _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
+    "sqa_attn_bwd_packed": (_I, [_P, _P, _I, _P, _P, _P, _I,
+                                 _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "sqa_attn_bwd_static": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I,
                                  _I, _I, _I, _I, _I, _I, _F, _P]),
     "sqa_proj": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
@@ -140,6 +143,14 @@ def sqa_attn_fwd_cross(q, k, v, out, out_dtype, lse, B, N_q, N_kv, H_q, H_kv, d_
                                         _stream(stream)), "sqa_attn_fwd_cross")
 
 
+def sqa_attn_fwd_packed(qkv, out, out_dtype, lse, B, N, H_q, H_kv, d_head, causal, scale,
+                        stream=None) -> None:
+    """Forward on a packed QKV buffer [B, N, H_q + 2*H_kv, d_head]."""
+    _check(library().sqa_attn_fwd_packed(_ptr(qkv), _ptr(out), int(out_dtype), _ptr(lse), B, N, H_q, H_kv,
+                                         d_head, int(bool(causal)), float(scale), _stream(stream)),
+           "sqa_attn_fwd_packed")
+
+
 def sqa_attn_bwd_workspace_size(B, N, H_q, H_kv, d_head) -> int:
     return int(library().sqa_attn_bwd_workspace_size(B, N, H_q, H_kv, d_head))
 
@@ -161,6 +172,15 @@ def sqa_attn_bwd_cross(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype,
                                         B, N_q, N_kv, H_q, H_kv, d_head, float(scale),
                                         _ptr(workspace), int(workspace_bytes), _stream(stream)),
            "sqa_attn_bwd_cross")
+
+
+def sqa_attn_bwd_packed(qkv, out, o_dtype, dout, lse, dqkv, grad_dtype, B, N, H_q, H_kv, d_head, causal,
+                        scale, workspace, workspace_bytes, stream=None) -> None:
+    """Gradient of sqa_attn_fwd_packed into a packed dQKV buffer."""
+    _check(library().sqa_attn_bwd_packed(_ptr(qkv), _ptr(out), int(o_dtype), _ptr(dout), _ptr(lse), _ptr(dqkv),
+                                         int(grad_dtype), B, N, H_q, H_kv, d_head, int(bool(causal)),
+                                         float(scale), _ptr(workspace), int(workspace_bytes), _stream(stream)),
+           "sqa_attn_bwd_packed")
 
 
 def sqa_attn_bwd_static(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B, N, H_q, H_kv,

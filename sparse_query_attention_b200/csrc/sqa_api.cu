@@ -83,6 +83,54 @@ sqa_status_t check_kv_length(int B, int N, int Nkv, int H_kv, int causal) {
   return SQA_OK;
 }
 
+// Shape, mask and token strides of one attention call.  A token stride is
+// the number of elements from one token's row of heads to the next: H * d for
+// the dense layouts, (H_q + 2 H_kv) * d inside a packed QKV buffer.
+struct AttnDesc {
+  int B, N, Nkv, H_q, H_kv, d, causal;
+  float scale;
+  long long ld_q, ld_kv;    // Q; K and V
+  long long ld_dq, ld_dkv;  // dQ; dK and dV (backward only)
+};
+
+AttnDesc dense_desc(int B, int N, int Nkv, int H_q, int H_kv, int d, int causal, float scale) {
+  AttnDesc a;
+  a.B = B;
+  a.N = N;
+  a.Nkv = Nkv;
+  a.H_q = H_q;
+  a.H_kv = H_kv;
+  a.d = d;
+  a.causal = causal ? 1 : 0;
+  a.scale = scale;
+  a.ld_q = a.ld_dq = static_cast<long long>(H_q) * d;
+  a.ld_kv = a.ld_dkv = static_cast<long long>(H_kv) * d;
+  return a;
+}
+
+// The packed layout [B, N, H_q + 2 H_kv, d]: Q heads, then K, then V.
+AttnDesc packed_desc(int B, int N, int H_q, int H_kv, int d, int causal, float scale) {
+  AttnDesc a = dense_desc(B, N, N, H_q, H_kv, d, causal, scale);
+  a.ld_q = a.ld_kv = a.ld_dq = a.ld_dkv = static_cast<long long>(H_q + 2 * H_kv) * d;
+  return a;
+}
+
+sqa_status_t check_desc(const void* q, const void* k, const void* v, const AttnDesc& a) {
+  sqa_status_t s = check_attn_args(q, k, v, a.B, a.N, a.H_q, a.H_kv, a.d, a.scale);
+  if (s != SQA_OK) return s;
+  s = check_kv_length(a.B, a.N, a.Nkv, a.H_kv, a.causal);
+  if (s != SQA_OK) return s;
+  // Token rows are whole 16-byte units (a TMA stride rule) and the element
+  // offsets of the last token of the last batch fit in 32-bit row arithmetic.
+  const long long lds[4] = {a.ld_q, a.ld_kv, a.ld_dq, a.ld_dkv};
+  for (long long ld : lds)
+    if (ld % 8 != 0) return SQA_ERR_INVALID_ARG;
+  if (a.ld_q < static_cast<long long>(a.H_q) * a.d || a.ld_dq < static_cast<long long>(a.H_q) * a.d ||
+      a.ld_kv < static_cast<long long>(a.H_kv) * a.d || a.ld_dkv < static_cast<long long>(a.H_kv) * a.d)
+    return SQA_ERR_INVALID_ARG;
+  return SQA_OK;
+}
+
 // ---------------------------------------------------------------------------
 // Attention forward
 // ---------------------------------------------------------------------------
@@ -99,9 +147,10 @@ int head_pack(int G) {
 }
 
 template <int D>
-sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* out, int out_bf16, float* lse, int B,
-                           int N, int Nkv, int H_q, int H_kv, int causal, float scale, cudaStream_t st) {
+sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* out, int out_bf16, float* lse,
+                           const AttnDesc& a, cudaStream_t st) {
   using C = sqa::FwdCfg<D>;
+  const int B = a.B, N = a.N, Nkv = a.Nkv, H_q = a.H_q, H_kv = a.H_kv;
   const int G = H_q / H_kv;
   const int g = head_pack(G);
   int log2g = 0;
@@ -111,13 +160,13 @@ sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* ou
   CUtensorMap mq, mk, mv;
   {
     const uint64_t dims[4] = {uint64_t(D), uint64_t(H_q), uint64_t(N), uint64_t(B)};
-    const uint64_t strides[3] = {uint64_t(D) * 2, uint64_t(H_q) * D * 2, uint64_t(N) * H_q * D * 2};
+    const uint64_t strides[3] = {uint64_t(D) * 2, uint64_t(a.ld_q) * 2, uint64_t(N) * a.ld_q * 2};
     const uint32_t box[4] = {uint32_t(C::kRowElems), uint32_t(g), uint32_t(T), 1};
     if (!make_map_bf16(&mq, q, 4, dims, strides, box, swz)) return SQA_ERR_CUDA;
   }
   {
     const uint64_t dims[4] = {uint64_t(D), uint64_t(H_kv), uint64_t(Nkv), uint64_t(B)};
-    const uint64_t strides[3] = {uint64_t(D) * 2, uint64_t(H_kv) * D * 2, uint64_t(Nkv) * H_kv * D * 2};
+    const uint64_t strides[3] = {uint64_t(D) * 2, uint64_t(a.ld_kv) * 2, uint64_t(Nkv) * a.ld_kv * 2};
     const uint32_t box[4] = {uint32_t(C::kRowElems), 1, 128, 1};
     if (!make_map_bf16(&mk, k, 4, dims, strides, box, swz)) return SQA_ERR_CUDA;
     if (!make_map_bf16(&mv, v, 4, dims, strides, box, swz)) return SQA_ERR_CUDA;
@@ -135,9 +184,9 @@ sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* ou
   p.log2g = log2g;
   p.n_sub = G / g;
   p.n_tblk = (N + 2 * T - 1) / (2 * T);
-  p.causal = causal ? 1 : 0;
+  p.causal = a.causal;
   p.out_bf16 = out_bf16;
-  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
   const long long gy = static_cast<long long>(H_kv) * p.n_sub;
   if (gy > 65535 || B > 65535) return SQA_ERR_UNSUPPORTED;
   auto kern = sqa::sqa_fwd_kernel<D>;
@@ -149,20 +198,18 @@ sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* ou
 }
 
 sqa_status_t attn_fwd_impl(const void* q, const void* k, const void* v, void* out, sqa_dtype_t out_dtype, float* lse,
-                           int B, int N, int Nkv, int H_q, int H_kv, int d, int causal, float scale, void* stream) {
-  sqa_status_t s = check_attn_args(q, k, v, B, N, H_q, H_kv, d, scale);
-  if (s != SQA_OK) return s;
-  s = check_kv_length(B, N, Nkv, H_kv, causal);
+                           const AttnDesc& a, void* stream) {
+  sqa_status_t s = check_desc(q, k, v, a);
   if (s != SQA_OK) return s;
   if (!out || !aligned16(out) || (lse && !aligned16(lse))) return SQA_ERR_INVALID_ARG;
   if (out_dtype != SQA_DT_F32 && out_dtype != SQA_DT_BF16) return SQA_ERR_INVALID_ARG;
   const int ob = out_dtype == SQA_DT_BF16;
   cudaStream_t st = as_stream(stream);
-  switch (d) {
-    case 16: return launch_fwd_tc<16>(q, k, v, out, ob, lse, B, N, Nkv, H_q, H_kv, causal, scale, st);
-    case 32: return launch_fwd_tc<32>(q, k, v, out, ob, lse, B, N, Nkv, H_q, H_kv, causal, scale, st);
-    case 64: return launch_fwd_tc<64>(q, k, v, out, ob, lse, B, N, Nkv, H_q, H_kv, causal, scale, st);
-    default: return launch_fwd_tc<128>(q, k, v, out, ob, lse, B, N, Nkv, H_q, H_kv, causal, scale, st);
+  switch (a.d) {
+    case 16: return launch_fwd_tc<16>(q, k, v, out, ob, lse, a, st);
+    case 32: return launch_fwd_tc<32>(q, k, v, out, ob, lse, a, st);
+    case 64: return launch_fwd_tc<64>(q, k, v, out, ob, lse, a, st);
+    default: return launch_fwd_tc<128>(q, k, v, out, ob, lse, a, st);
   }
 }
 
@@ -192,20 +239,22 @@ bool make_map_f32_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_
 }
 
 // bf16 [B, N, H, D] viewed as the 4-D map {D, H, N, B}, box {row, heads, tokens, 1}.
+// ld: elements from one token to the next (H * D when dense).
 template <int D>
-bool make_map_bnhd(CUtensorMap* map, const void* base, int B, int N, int H, uint32_t box_heads,
+bool make_map_bnhd(CUtensorMap* map, const void* base, int B, int N, int H, long long ld, uint32_t box_heads,
                    uint32_t box_tokens) {
   constexpr int kRowElems = D < 64 ? D : 64;
   const uint64_t dims[4] = {uint64_t(D), uint64_t(H), uint64_t(N), uint64_t(B)};
-  const uint64_t strides[3] = {uint64_t(D) * 2, uint64_t(H) * D * 2, uint64_t(N) * H * D * 2};
+  const uint64_t strides[3] = {uint64_t(D) * 2, uint64_t(ld) * 2, uint64_t(N) * ld * 2};
   const uint32_t box[4] = {uint32_t(kRowElems), box_heads, box_tokens, 1};
   return make_map_bf16(map, base, 4, dims, strides, box, tma_swizzle_for_row_bytes(kRowElems * 2));
 }
 
 template <int D, typename GradT>
 sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const void* o, int o_bf16, const void* dout,
-                           const float* lse, void* dq, void* dk, void* dv, int B, int N, int Nkv, int H_q,
-                           int H_kv, int causal, float scale, void* workspace, cudaStream_t st) {
+                           const float* lse, void* dq, void* dk, void* dv, const AttnDesc& a, void* workspace,
+                           cudaStream_t st) {
+  const int B = a.B, N = a.N, Nkv = a.Nkv, H_q = a.H_q, H_kv = a.H_kv;
   const int n_pad = bwd_n_pad(N);
   float* dsum = static_cast<float*>(workspace);
   float* lse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + bwd_half_bytes(B, N, H_q));
@@ -232,17 +281,23 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
   p.log2g = log2g;
   p.n_sub = G / g;
   p.n_tblk = (N + T - 1) / T;
-  p.causal = causal ? 1 : 0;
-  p.scale = scale;
-  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = a.causal;
+  p.scale = a.scale;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.ld_dq = static_cast<int>(a.ld_dq);
+  p.ld_dkv = static_cast<int>(a.ld_dkv);
   const long long gy = static_cast<long long>(H_kv) * p.n_sub;
   if (gy > 65535 || B > 65535) return SQA_ERR_UNSUPPORTED;
 
   CUtensorMap m_k128, m_v128, m_q64, m_do64, m_l2, m_ds, m_qp, m_dop, m_k64, m_v64;
-  if (!make_map_bnhd<D>(&m_k128, k, B, Nkv, H_kv, 1, 128) || !make_map_bnhd<D>(&m_v128, v, B, Nkv, H_kv, 1, 128) ||
-      !make_map_bnhd<D>(&m_q64, q, B, N, H_q, 1, 64) || !make_map_bnhd<D>(&m_do64, dout, B, N, H_q, 1, 64) ||
-      !make_map_bnhd<D>(&m_qp, q, B, N, H_q, g, T) || !make_map_bnhd<D>(&m_dop, dout, B, N, H_q, g, T) ||
-      !make_map_bnhd<D>(&m_k64, k, B, Nkv, H_kv, 1, 64) || !make_map_bnhd<D>(&m_v64, v, B, Nkv, H_kv, 1, 64) ||
+  const long long ld_do = static_cast<long long>(H_q) * D;  // dO is always dense
+  if (!make_map_bnhd<D>(&m_k128, k, B, Nkv, H_kv, a.ld_kv, 1, 128) ||
+      !make_map_bnhd<D>(&m_v128, v, B, Nkv, H_kv, a.ld_kv, 1, 128) ||
+      !make_map_bnhd<D>(&m_q64, q, B, N, H_q, a.ld_q, 1, 64) ||
+      !make_map_bnhd<D>(&m_do64, dout, B, N, H_q, ld_do, 1, 64) ||
+      !make_map_bnhd<D>(&m_qp, q, B, N, H_q, a.ld_q, g, T) || !make_map_bnhd<D>(&m_dop, dout, B, N, H_q, ld_do, g, T) ||
+      !make_map_bnhd<D>(&m_k64, k, B, Nkv, H_kv, a.ld_kv, 1, 64) ||
+      !make_map_bnhd<D>(&m_v64, v, B, Nkv, H_kv, a.ld_kv, 1, 64) ||
       !make_map_f32_2d(&m_l2, lse2, n_pad, uint64_t(B) * H_q, 64) ||
       !make_map_f32_2d(&m_ds, dsum, n_pad, uint64_t(B) * H_q, 64))
     return SQA_ERR_CUDA;
@@ -277,22 +332,17 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
 
 template <int D>
 sqa_status_t launch_bwd_d(bool grad_bf16, const void* q, const void* k, const void* v, const void* o, int o_bf16,
-                          const void* dout, const float* lse, void* dq, void* dk, void* dv, int B, int N, int Nkv,
-                          int H_q, int H_kv, int causal, float scale, void* ws, cudaStream_t st) {
+                          const void* dout, const float* lse, void* dq, void* dk, void* dv, const AttnDesc& a,
+                          void* ws, cudaStream_t st) {
   if (grad_bf16)
-    return launch_bwd_tc<D, __nv_bfloat16>(q, k, v, o, o_bf16, dout, lse, dq, dk, dv, B, N, Nkv, H_q, H_kv, causal,
-                                           scale, ws, st);
-  return launch_bwd_tc<D, float>(q, k, v, o, o_bf16, dout, lse, dq, dk, dv, B, N, Nkv, H_q, H_kv, causal, scale, ws,
-                                 st);
+    return launch_bwd_tc<D, __nv_bfloat16>(q, k, v, o, o_bf16, dout, lse, dq, dk, dv, a, ws, st);
+  return launch_bwd_tc<D, float>(q, k, v, o, o_bf16, dout, lse, dq, dk, dv, a, ws, st);
 }
 
 sqa_status_t attn_bwd_impl(const void* q, const void* k, const void* v, const void* out, sqa_dtype_t o_dtype,
                            const void* dout, const float* lse, void* dq, void* dk, void* dv, sqa_dtype_t grad_dtype,
-                           int B, int N, int Nkv, int H_q, int H_kv, int d_head, int causal, float scale,
-                           void* workspace, size_t workspace_bytes, void* stream) {
-  sqa_status_t s = check_attn_args(q, k, v, B, N, H_q, H_kv, d_head, scale);
-  if (s != SQA_OK) return s;
-  s = check_kv_length(B, N, Nkv, H_kv, causal);
+                           const AttnDesc& a, void* workspace, size_t workspace_bytes, void* stream) {
+  sqa_status_t s = check_desc(q, k, v, a);
   if (s != SQA_OK) return s;
   if (!out || !dout || !lse || !dq || !dk || !dv || !workspace) return SQA_ERR_INVALID_ARG;
   if (!aligned16(out) || !aligned16(dout) || !aligned16(lse) || !aligned16(dq) || !aligned16(dk) ||
@@ -300,23 +350,15 @@ sqa_status_t attn_bwd_impl(const void* q, const void* k, const void* v, const vo
     return SQA_ERR_INVALID_ARG;
   if ((o_dtype != SQA_DT_F32 && o_dtype != SQA_DT_BF16) || (grad_dtype != SQA_DT_F32 && grad_dtype != SQA_DT_BF16))
     return SQA_ERR_INVALID_ARG;
-  if (workspace_bytes < bwd_workspace_bytes(B, N, H_q)) return SQA_ERR_INVALID_ARG;
+  if (workspace_bytes < bwd_workspace_bytes(a.B, a.N, a.H_q)) return SQA_ERR_INVALID_ARG;
   const bool gb = grad_dtype == SQA_DT_BF16;
   const int ob = o_dtype == SQA_DT_BF16;
   cudaStream_t st = as_stream(stream);
-  switch (d_head) {
-    case 16:
-      return launch_bwd_d<16>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, Nkv, H_q, H_kv, causal, scale,
-                              workspace, st);
-    case 32:
-      return launch_bwd_d<32>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, Nkv, H_q, H_kv, causal, scale,
-                              workspace, st);
-    case 64:
-      return launch_bwd_d<64>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, Nkv, H_q, H_kv, causal, scale,
-                              workspace, st);
-    default:
-      return launch_bwd_d<128>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, B, N, Nkv, H_q, H_kv, causal, scale,
-                               workspace, st);
+  switch (a.d) {
+    case 16: return launch_bwd_d<16>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, a, workspace, st);
+    case 32: return launch_bwd_d<32>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, a, workspace, st);
+    case 64: return launch_bwd_d<64>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, a, workspace, st);
+    default: return launch_bwd_d<128>(gb, q, k, v, out, ob, dout, lse, dq, dk, dv, a, workspace, st);
   }
 }
 
@@ -389,25 +431,42 @@ sqa_status_t gemm_impl(const void* a, bool a_mn, const void* b, bool b_mn, const
             : launch_gemm_layouts<false, true, false>(ma, mb, bn, bias, c, M, N, K, accumulate, st);
 }
 
+// Byte offset of head `h` within one token row of d-element heads.
+inline const void* head_ptr(const void* base, int h, int d, size_t elem) {
+  return base ? static_cast<const uint8_t*>(base) + static_cast<size_t>(h) * d * elem : nullptr;
+}
+inline void* head_ptr(void* base, int h, int d, size_t elem) {
+  return base ? static_cast<uint8_t*>(base) + static_cast<size_t>(h) * d * elem : nullptr;
+}
+
 }  // namespace
 
 extern "C" {
 
 sqa_status_t sqa_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int N, int H_q, int H_kv,
                           int d_head, int causal, float scale, void* stream) {
-  return attn_fwd_impl(q, k, v, out, SQA_DT_F32, nullptr, B, N, N, H_q, H_kv, d_head, causal, scale, stream);
+  return attn_fwd_impl(q, k, v, out, SQA_DT_F32, nullptr, dense_desc(B, N, N, H_q, H_kv, d_head, causal, scale),
+                       stream);
 }
 
 sqa_status_t sqa_attn_fwd_ex(const void* q, const void* k, const void* v, void* out, sqa_dtype_t out_dtype,
                              float* lse, int B, int N, int H_q, int H_kv, int d_head, int causal, float scale,
                              void* stream) {
-  return attn_fwd_impl(q, k, v, out, out_dtype, lse, B, N, N, H_q, H_kv, d_head, causal, scale, stream);
+  return attn_fwd_impl(q, k, v, out, out_dtype, lse, dense_desc(B, N, N, H_q, H_kv, d_head, causal, scale), stream);
 }
 
 sqa_status_t sqa_attn_fwd_cross(const void* q, const void* k, const void* v, void* out, sqa_dtype_t out_dtype,
                                 float* lse, int B, int N_q, int N_kv, int H_q, int H_kv, int d_head, float scale,
                                 void* stream) {
-  return attn_fwd_impl(q, k, v, out, out_dtype, lse, B, N_q, N_kv, H_q, H_kv, d_head, 0, scale, stream);
+  return attn_fwd_impl(q, k, v, out, out_dtype, lse, dense_desc(B, N_q, N_kv, H_q, H_kv, d_head, 0, scale),
+                       stream);
+}
+
+sqa_status_t sqa_attn_fwd_packed(const void* qkv, void* out, sqa_dtype_t out_dtype, float* lse, int B, int N,
+                                 int H_q, int H_kv, int d_head, int causal, float scale, void* stream) {
+  if (H_q <= 0 || H_kv <= 0 || d_head <= 0 || H_q > (1 << 20) || H_kv > (1 << 20)) return SQA_ERR_INVALID_ARG;
+  return attn_fwd_impl(qkv, head_ptr(qkv, H_q, d_head, 2), head_ptr(qkv, H_q + H_kv, d_head, 2), out, out_dtype,
+                       lse, packed_desc(B, N, H_q, H_kv, d_head, causal, scale), stream);
 }
 
 size_t sqa_attn_bwd_workspace_size(int B, int N, int H_q, int H_kv, int d_head) {
@@ -419,16 +478,29 @@ sqa_status_t sqa_attn_bwd(const void* q, const void* k, const void* v, const voi
                           const void* dout, const float* lse, void* dq, void* dk, void* dv, sqa_dtype_t grad_dtype,
                           int B, int N, int H_q, int H_kv, int d_head, int causal, float scale, void* workspace,
                           size_t workspace_bytes, void* stream) {
-  return attn_bwd_impl(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B, N, N, H_q, H_kv, d_head, causal,
-                       scale, workspace, workspace_bytes, stream);
+  return attn_bwd_impl(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype,
+                       dense_desc(B, N, N, H_q, H_kv, d_head, causal, scale), workspace, workspace_bytes, stream);
 }
 
 sqa_status_t sqa_attn_bwd_cross(const void* q, const void* k, const void* v, const void* out, sqa_dtype_t o_dtype,
                                 const void* dout, const float* lse, void* dq, void* dk, void* dv,
                                 sqa_dtype_t grad_dtype, int B, int N_q, int N_kv, int H_q, int H_kv, int d_head,
                                 float scale, void* workspace, size_t workspace_bytes, void* stream) {
-  return attn_bwd_impl(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B, N_q, N_kv, H_q, H_kv, d_head, 0,
-                       scale, workspace, workspace_bytes, stream);
+  return attn_bwd_impl(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype,
+                       dense_desc(B, N_q, N_kv, H_q, H_kv, d_head, 0, scale), workspace, workspace_bytes, stream);
+}
+
+sqa_status_t sqa_attn_bwd_packed(const void* qkv, const void* out, sqa_dtype_t o_dtype, const void* dout,
+                                 const float* lse, void* dqkv, sqa_dtype_t grad_dtype, int B, int N, int H_q,
+                                 int H_kv, int d_head, int causal, float scale, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (H_q <= 0 || H_kv <= 0 || d_head <= 0 || H_q > (1 << 20) || H_kv > (1 << 20)) return SQA_ERR_INVALID_ARG;
+  if (grad_dtype != SQA_DT_F32 && grad_dtype != SQA_DT_BF16) return SQA_ERR_INVALID_ARG;
+  const size_t ge = grad_dtype == SQA_DT_BF16 ? 2 : 4;
+  return attn_bwd_impl(qkv, head_ptr(qkv, H_q, d_head, 2), head_ptr(qkv, H_q + H_kv, d_head, 2), out, o_dtype,
+                       dout, lse, dqkv, head_ptr(dqkv, H_q, d_head, ge), head_ptr(dqkv, H_q + H_kv, d_head, ge),
+                       grad_dtype, packed_desc(B, N, H_q, H_kv, d_head, causal, scale), workspace, workspace_bytes,
+                       stream);
 }
 
 }  // extern "C"

@@ -118,6 +118,7 @@ struct BwdParams {
   const float* lse2;  // [B, H_q, n_pad]
   int B, N, H_q, H_kv, G, n_pad;  // N: query tokens, n_pad: N rounded up to 128
   int Nkv;                        // key/value tokens (N for self-attention)
+  int ld_dq, ld_dkv;              // token strides (elements) of dQ and of dK/dV
   int g, log2g, n_sub, n_tblk;  // packing of the dQ kernel
   int causal;
   float scale;
@@ -381,7 +382,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t col = grp == 0 ? C::kColDV : C::kColDK;
       const float mult = grp == 0 ? 1.f : p.scale;
       GradT* dst = static_cast<GradT*>(grp == 0 ? p.dv : p.dk) +
-                   ((static_cast<size_t>(b) * p.Nkv + (valid ? u : 0)) * p.H_kv + j) * D;
+                   (static_cast<size_t>(b) * p.Nkv + (valid ? u : 0)) * p.ld_dkv + static_cast<size_t>(j) * D;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 16) {
         uint32_t rr[16];
@@ -627,7 +628,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (ok) {
       tc_fence_after();
       const bool valid = tok < p.N;
-      GradT* dst = static_cast<GradT*>(p.dq) + ((static_cast<size_t>(b) * p.N + (valid ? tok : 0)) * p.H_q + head) * D;
+      GradT* dst = static_cast<GradT*>(p.dq) + (static_cast<size_t>(b) * p.N + (valid ? tok : 0)) * p.ld_dq +
+                   static_cast<size_t>(head) * D;
       // The two groups split the columns of dQ (group 0 alone when D = 16).
       constexpr int kHalf = D >= 32 ? D / 2 : D;
 #pragma unroll 1
