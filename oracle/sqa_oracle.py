@@ -17,6 +17,11 @@ What it restates, and from where:
   "ReactiveAI/GQA-Ref-Micro" model card, note on model size.)
 * Causal masking for the decoder models (the training/inference usage on
   both model cards) and no mask for encoder-style work (abstract).
+* Sliding-window (local) attention, the spatially sparse pattern SQA is
+  set beside ("ReactiveAI/GQA-Ref-Micro" model card, results paragraph: SQA
+  as a possible alternative to spatially sparse attention; the paper's
+  "Builds on" list includes Longformer): query t sees keys
+  t - left <= u <= t + right, optionally together with the causal mask.
 
 The pages print no equations, so the attention itself is the textbook
 definition that "extension to Grouped Query Attention" presupposes.  Readings
@@ -56,8 +61,22 @@ def _check_lengths(N_q: int, N_kv: int, causal: bool) -> None:
         raise ValueError("causal attention needs as many keys as queries")
 
 
-def _scores(q_rows, k_head, t_rows, causal, scale):
-    """s[r, u] = scale * <q_r, k_u>, with u > t_r set to -inf when causal.
+def _check_window(window, N_q: int, N_kv: int):
+    # A window relates query and key positions of one sequence.
+    if window is None:
+        return None
+    left, right = (int(w) for w in window)
+    if left < 0 or right < 0:
+        raise ValueError("window sides must be >= 0")
+    if N_q != N_kv:
+        raise ValueError("a window needs as many keys as queries")
+    return left, right
+
+
+def _scores(q_rows, k_head, t_rows, causal, scale, window=None):
+    """s[r, u] = scale * <q_r, k_u>, set to -inf where key u is hidden from
+    query t_r: u > t_r when causal; u < t_r - left or u > t_r + right for a
+    window (left, right).
 
     Only keys 0..max(t_rows) can be unmasked in the causal case, so the
     columns beyond are never formed; masked entries inside are -inf.
@@ -66,19 +85,26 @@ def _scores(q_rows, k_head, t_rows, causal, scale):
         n_keys = int(t_rows.max()) + 1
         k_head = k_head[:n_keys]
     s = scale * (q_rows @ k_head.T)
+    u = np.arange(k_head.shape[0])
     if causal:
-        u = np.arange(k_head.shape[0])
         s[u[None, :] > t_rows[:, None]] = -np.inf
+    if window is not None:
+        left, right = window
+        s[u[None, :] < t_rows[:, None] - left] = -np.inf
+        s[u[None, :] > t_rows[:, None] + right] = -np.inf
     return s, k_head.shape[0]
 
 
-def attention_forward(q, k, v, causal: bool, scale: float, rows=None):
+def attention_forward(q, k, v, causal: bool, scale: float, rows=None, window=None):
     """Sparse Query Attention output and log-sum-exp.
 
     q: [B, N, H_q, d]; k, v: [B, N_kv, H_kv, d] (float64 arrays; N_kv = N
     for self-attention, any length for cross / memory attention, which is
     never causal).
     rows: optional 1-D array of query token indices; all rows when None.
+    window: optional (left, right): query t sees only keys
+    t - left <= u <= t + right (self-attention only; every row keeps at
+    least key t).
     Returns o [B, R, H_q, d] and lse [B, H_q, R] (R = number of rows), with
         o[b,t,h]   = sum_u softmax_u(s_tu) v[b,u,j],  j = h // G
         lse[b,h,t] = log sum_u exp(s_tu)
@@ -90,6 +116,7 @@ def attention_forward(q, k, v, causal: bool, scale: float, rows=None):
     H_kv = k.shape[2]
     G = _check_heads(H_q, H_kv)
     _check_lengths(N, k.shape[1], causal)
+    window = _check_window(window, N, k.shape[1])
     t_all = np.arange(N) if rows is None else np.asarray(rows, dtype=np.int64)
     R = t_all.shape[0]
     o = np.empty((B, R, H_q, d), dtype=np.float64)
@@ -99,7 +126,7 @@ def attention_forward(q, k, v, causal: bool, scale: float, rows=None):
             j = h // G
             for c0 in range(0, R, _CHUNK):
                 t = t_all[c0:c0 + _CHUNK]
-                s, n_keys = _scores(q[b, t, h, :], k[b, :, j, :], t, causal, scale)
+                s, n_keys = _scores(q[b, t, h, :], k[b, :, j, :], t, causal, scale, window)
                 m = s.max(axis=1, keepdims=True)
                 w = np.exp(s - m)
                 l = w.sum(axis=1)
@@ -108,7 +135,7 @@ def attention_forward(q, k, v, causal: bool, scale: float, rows=None):
     return o, lse
 
 
-def attention_backward(q, k, v, do, causal: bool, scale: float):
+def attention_backward(q, k, v, do, causal: bool, scale: float, window=None):
     """Gradients of L = sum(o * do) with respect to q, k and v.
 
     Chain rule through the definition above, per (b, h) with j = h // G:
@@ -118,6 +145,7 @@ def attention_backward(q, k, v, do, causal: bool, scale: float):
         dq_h  = scale * dS k_j
         dk_j += scale * dS^T q_h             (summed over the G heads of group j)
         dv_j += P^T do_h                     (summed over the G heads of group j)
+    with P zero outside the causal mask / window, as in attention_forward.
     Returns dq [B,N,H_q,d], dk and dv [B,N,H_kv,d].
     """
     q = np.asarray(q, dtype=np.float64)
@@ -128,6 +156,7 @@ def attention_backward(q, k, v, do, causal: bool, scale: float):
     H_kv = k.shape[2]
     G = _check_heads(H_q, H_kv)
     _check_lengths(N, k.shape[1], causal)
+    window = _check_window(window, N, k.shape[1])
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
@@ -137,7 +166,7 @@ def attention_backward(q, k, v, do, causal: bool, scale: float):
             j = h // G
             for c0 in range(0, N, _CHUNK):
                 t = t_all[c0:c0 + _CHUNK]
-                s, n_keys = _scores(q[b, t, h, :], k[b, :, j, :], t, causal, scale)
+                s, n_keys = _scores(q[b, t, h, :], k[b, :, j, :], t, causal, scale, window)
                 m = s.max(axis=1, keepdims=True)
                 w = np.exp(s - m)
                 p = w / w.sum(axis=1, keepdims=True)

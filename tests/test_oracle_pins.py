@@ -446,3 +446,111 @@ def test_rejects_bad_head_counts():
     k = np.zeros((1, 2, 2, 4))
     with pytest.raises(ValueError):
         attention_forward(q, k, k, False, 1.0)
+
+
+# ---------------------------------------------------------------------------
+# Sliding-window (local) attention
+# ---------------------------------------------------------------------------
+def brute_attention_window(q, k, v, scale, left, right, causal=False):
+    """fsum brute force; the visible keys of query t are listed explicitly:
+    max(0, t - left) .. min(N - 1, t + right), capped at t when causal."""
+    B, N, H_q, d = q.shape
+    G = H_q // k.shape[2]
+    o = np.zeros(q.shape)
+    lse = np.zeros((B, H_q, N))
+    for b in range(B):
+        for h in range(H_q):
+            for t in range(N):
+                last = min(N - 1, t + right)
+                if causal:
+                    last = min(last, t)
+                keys = list(range(max(0, t - left), last + 1))
+                e = [math.exp(scale * math.fsum(q[b, t, h, c] * k[b, u, h // G, c] for c in range(d))) for u in keys]
+                z = math.fsum(e)
+                for c in range(d):
+                    o[b, t, h, c] = math.fsum(e[i] * v[b, u, h // G, c] for i, u in enumerate(keys)) / z
+                lse[b, h, t] = math.log(z)
+    return o, lse
+
+
+@pytest.mark.parametrize("left,right,causal", [(2, 0, False), (1, 3, False), (0, 0, False), (3, 3, True),
+                                               (9, 9, False)])
+def test_window_brute_force(left, right, causal):
+    rng = np.random.default_rng(left * 10 + right)
+    B, N, H_q, H_kv, d = 1, 7, 4, 2, 3
+    q, k, v = _rand((B, N, H_q, d), rng), _rand((B, N, H_kv, d), rng), _rand((B, N, H_kv, d), rng)
+    o, lse = attention_forward(q, k, v, causal, 0.7, window=(left, right))
+    ob, lb = brute_attention_window(q, k, v, 0.7, left, right, causal)
+    np.testing.assert_allclose(o, ob, atol=1e-12)
+    np.testing.assert_allclose(lse, lb, atol=1e-12)
+
+
+def _band_mask(N, left, right):
+    t = torch.arange(N)[:, None]
+    u = torch.arange(N)[None, :]
+    return (u >= t - left) & (u <= t + right)
+
+
+@pytest.mark.parametrize("left,right,heads", [(4, 0, (4, 2)), (2, 5, (4, 4)), (0, 6, (8, 1))])
+def test_window_matches_sdpa_mask_and_autograd(left, right, heads):
+    """The window as an explicit boolean mask handed to torch SDPA (fp64):
+    output, and all three gradients through autograd."""
+    H_q, H_kv = heads
+    rng = np.random.default_rng(100 + left + 7 * right)
+    B, N, d = 2, 13, 8
+    q, k, v = _rand((B, N, H_q, d), rng), _rand((B, N, H_kv, d), rng), _rand((B, N, H_kv, d), rng)
+    do = _rand((B, N, H_q, d), rng)
+    scale = 1 / math.sqrt(d)
+    o, _ = attention_forward(q, k, v, False, scale, window=(left, right))
+    tq, tk, tv = (torch.from_numpy(a.copy()).permute(0, 2, 1, 3).requires_grad_() for a in (q, k, v))
+    to = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=_band_mask(N, left, right), scale=scale,
+                                        enable_gqa=H_q != H_kv)
+    np.testing.assert_allclose(o, to.detach().permute(0, 2, 1, 3).numpy(), atol=1e-12)
+    to.backward(torch.from_numpy(do).permute(0, 2, 1, 3))
+    dq, dk, dv = attention_backward(q, k, v, do, False, scale, window=(left, right))
+    np.testing.assert_allclose(dq, tq.grad.permute(0, 2, 1, 3).numpy(), atol=1e-12)
+    np.testing.assert_allclose(dk, tk.grad.permute(0, 2, 1, 3).numpy(), atol=1e-12)
+    np.testing.assert_allclose(dv, tv.grad.permute(0, 2, 1, 3).numpy(), atol=1e-12)
+
+
+def test_window_degenerate_cases():
+    """(0, 0): each token sees only itself, so O = V of its own token, LSE is
+    its own scaled score, and dQ = dK = 0 with dV = the group sum of dO.
+    (N, 0) is the causal mask and (N, N) no mask at all."""
+    rng = np.random.default_rng(8)
+    B, N, H_q, H_kv, d = 2, 9, 4, 2, 5
+    q, k, v = _rand((B, N, H_q, d), rng), _rand((B, N, H_kv, d), rng), _rand((B, N, H_kv, d), rng)
+    do = _rand((B, N, H_q, d), rng)
+    o, lse = attention_forward(q, k, v, False, 0.3, window=(0, 0))
+    kx, vx = np.repeat(k, 2, axis=2), np.repeat(v, 2, axis=2)
+    np.testing.assert_allclose(o, vx, atol=1e-14)
+    np.testing.assert_allclose(lse, 0.3 * np.einsum("bthc,bthc->bht", q, kx), atol=1e-13)
+    dq, dk, dv = attention_backward(q, k, v, do, False, 0.3, window=(0, 0))
+    np.testing.assert_allclose(dq, 0, atol=1e-14)
+    np.testing.assert_allclose(dk, 0, atol=1e-14)
+    np.testing.assert_allclose(dv, do.reshape(B, N, H_kv, 2, d).sum(axis=3), atol=1e-14)
+    for win, causal in (((N, 0), True), ((N, N), False)):
+        ow, lw = attention_forward(q, k, v, False, 0.3, window=win)
+        oc, lc = attention_forward(q, k, v, causal, 0.3)
+        np.testing.assert_allclose(ow, oc, atol=1e-13)
+        np.testing.assert_allclose(lw, lc, atol=1e-13)
+
+
+def test_window_gradient_invariants():
+    """Softmax rows still sum to one inside the window: sum_u dK = 0 per KV
+    head and sum_u dV = sum of dO over the group's heads and all tokens."""
+    rng = np.random.default_rng(12)
+    B, N, H_q, H_kv, d = 1, 11, 6, 2, 4
+    q, k, v = _rand((B, N, H_q, d), rng), _rand((B, N, H_kv, d), rng), _rand((B, N, H_kv, d), rng)
+    do = _rand((B, N, H_q, d), rng)
+    dq, dk, dv = attention_backward(q, k, v, do, False, 0.5, window=(3, 1))
+    np.testing.assert_allclose(dk.sum(axis=1), 0, atol=1e-12)
+    np.testing.assert_allclose(dv.sum(axis=1), do.reshape(B, N, H_kv, 3, d).sum(axis=(1, 3)), atol=1e-12)
+
+
+def test_window_rejects_bad_arguments():
+    z = np.zeros((1, 4, 1, 2))
+    with pytest.raises(ValueError):
+        attention_forward(z, z, z, False, 1.0, window=(-1, 0))
+    with pytest.raises(ValueError):
+        attention_forward(z, np.zeros((1, 5, 1, 2)), np.zeros((1, 5, 1, 2)), False, 1.0, window=(2, 2))
