@@ -250,6 +250,81 @@ def time_long_sequences(sqa, torch, stream, dev, reps=3):
     return {"config": {"B": 1, "d_head": d, "causal": False}, "by_N": res}
 
 
+WINDOW = {"B": 1, "N": 131072, "d_head": 128, "windows": {"causal_4096": (4095, 0), "local_2048": (2048, 2048)}}
+
+
+def window_pairs(N, left, right):
+    """Visible (query, key) pairs of a band t - left <= u <= t + right:
+    the sum over t of min(N - 1, t + right) - max(0, t - left) + 1."""
+    import numpy as np
+
+    t = np.arange(N, dtype=np.int64)
+    return int((np.minimum(N - 1, t + right) - np.maximum(0, t - left) + 1).sum())
+
+
+def time_windowed(sqa, torch, stream, dev, reps=3):
+    """Sliding-window SQA at N = 131072 (B=1, d=128): a causal window of 4096
+    keys and a symmetric local window of +-2048, forward for MHA, SQA and
+    xSQA on the same kernel, and the SQA training step (forward + backward)
+    with the causal window.  FLOPs count visible pairs only
+    (4 * H_q * P_w * d forward, 8 * H_q * P_w * d backward), so a rate close
+    to the dense kernel's means the skipped tiles cost nothing."""
+    from sqa_inputs import attention_inputs
+
+    c = WINDOW
+    N, d = c["N"], c["d_head"]
+    sc = 1 / math.sqrt(d)
+
+    def med(fn):
+        fn()
+        times = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        return statistics.median(times)
+
+    res = {}
+    for wname, (left, right) in c["windows"].items():
+        P_w = window_pairs(N, left, right)
+        per = {}
+        for name, (hq, hkv) in LONG_VARIANTS.items():
+            x = attention_inputs(1, N, hq, hkv, d, seed=3, device=dev)
+            o = torch.empty((1, N, hq, d), dtype=torch.float32, device=dev)
+            ms = med(lambda: sqa.sqa_attn_fwd_window(x["q"], x["k"], x["v"], o, sqa.SQA_DT_F32, None, 1, N, hq, hkv,
+                                                     d, left, right, sc, stream=stream))
+            per[name] = {"H_q": hq, "H_kv": hkv, "ms": ms, "tflops": 4 * hq * P_w * d / ms / 1e9,
+                         "tokens_per_s": N / (ms / 1e3)}
+            del x, o
+        for name in per:
+            per[name]["speedup_vs_mha"] = per["MHA"]["ms"] / per[name]["ms"]
+        res[wname] = {"left": left, "right": right, "visible_pairs": P_w, "forward": per}
+    # SQA training step with the causal window.
+    left, right = c["windows"]["causal_4096"]
+    hq, hkv = LONG_VARIANTS["SQA"]
+    P_w = window_pairs(N, left, right)
+    x = attention_inputs(1, N, hq, hkv, d, seed=3, with_dout=True, device=dev)
+    o = torch.empty((1, N, hq, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((1, hq, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty(t.shape, dtype=torch.bfloat16, device=dev) for t in (x["q"], x["k"], x["v"]))
+    wsb = sqa.sqa_attn_bwd_workspace_size(1, N, hq, hkv, d)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    BF = sqa.SQA_DT_BF16
+    fwd_ms = med(lambda: sqa.sqa_attn_fwd_window(x["q"], x["k"], x["v"], o, BF, lse, 1, N, hq, hkv, d, left, right,
+                                                 sc, stream=stream))
+    bwd_ms = med(lambda: sqa.sqa_attn_bwd_window(x["q"], x["k"], x["v"], o, BF, x["do"], lse, dq, dk, dv, BF, 1, N,
+                                                 hq, hkv, d, left, right, sc, ws, wsb, stream=stream))
+    res["sqa_train_causal_4096"] = {"fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+                                    "fwd_tflops": 4 * hq * P_w * d / fwd_ms / 1e9,
+                                    "bwd_tflops": 8 * hq * P_w * d / bwd_ms / 1e9,
+                                    "tokens_per_s": N / ((fwd_ms + bwd_ms) / 1e3)}
+    sqa.sqa_device_status(stream)
+    return {"config": {"B": 1, "N": N, "d_head": d}, "windows": res}
+
+
 LAYER = {"B": 16, "N": 1024, "d_model": 256, "d_head": 16, "causal": True}
 LAYER_VARIANTS = {"MHA": (16, 16), "GQA": (16, 4), "SQA": (8, 4), "sSQA": (8, 8), "xSQA": (4, 4), "xSMQA": (4, 1)}
 
@@ -495,6 +570,7 @@ def run_sqa(args):
     training = time_training_step(sqa, torch, stream, flush, dev)
     layer = time_decoder_layer(sqa, torch, stream, flush, dev)
     long_seq = time_long_sequences(sqa, torch, stream, dev)
+    windowed = time_windowed(sqa, torch, stream, dev)
 
     peak, peak_kind = load_peaks()
     achieved = flops_step / (statistics.mean(per_launch_ms) / 1e3) / 1e12
@@ -516,6 +592,7 @@ def run_sqa(args):
         "training_step": training,
         "decoder_layer": layer,
         "long_sequences": long_seq,
+        "windowed": windowed,
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -139,6 +139,38 @@ sqa_status_t sqa_attn_bwd_cross(const void* q, const void* k, const void* v,
                                 void* stream);
 
 /*
+ * sqa_attn_fwd_window - sliding-window (local) SQA: query t attends only to
+ * the keys u with t - window_left <= u <= t + window_right (and u < N).
+ * Spatially sparse attention of this kind is what the GQA-Ref-Micro model
+ * card (results paragraph) sets SQA beside; the paper's "Builds on" list
+ * includes Longformer.  The query-head reduction and the band combine: the
+ * cost is 4 * B * H_q * P_w * d FLOPs, P_w = number of visible (t, u) pairs.
+ * Common forms: a causal window of W keys is (W - 1, 0); a symmetric local
+ * window is (w, w).  A side of N or more is unbounded, so (N, 0) is the
+ * causal mask and (N, N) no mask.  Key tiles outside every row's band are
+ * skipped, not masked.
+ * Self-attention only (K/V have N tokens); window_left, window_right >= 0
+ * (else SQA_ERR_INVALID_ARG).  Layouts, dtypes and lse as sqa_attn_fwd_ex.
+ */
+sqa_status_t sqa_attn_fwd_window(const void* q, const void* k, const void* v, void* out,
+                                 sqa_dtype_t out_dtype, float* lse,
+                                 int B, int N, int H_q, int H_kv, int d_head,
+                                 int window_left, int window_right, float scale, void* stream);
+
+/*
+ * sqa_attn_bwd_window - gradient of sqa_attn_fwd_window (same window);
+ * arguments otherwise as sqa_attn_bwd, workspace from
+ * sqa_attn_bwd_workspace_size(B, N, H_q, H_kv, d_head).
+ */
+sqa_status_t sqa_attn_bwd_window(const void* q, const void* k, const void* v,
+                                 const void* out, sqa_dtype_t o_dtype,
+                                 const void* dout, const float* lse,
+                                 void* dq, void* dk, void* dv, sqa_dtype_t grad_dtype,
+                                 int B, int N, int H_q, int H_kv, int d_head,
+                                 int window_left, int window_right, float scale,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * sqa_attn_fwd_packed - the forward on a packed QKV buffer, the output of one
  * fused input projection with the concatenated weight [Wq; Wk; Wv]
  * ((H_q + 2 H_kv) * d_head rows): qkv [B, N, H_q + 2 H_kv, d_head] bf16,

@@ -35,12 +35,15 @@ SIGNATURES = {
     "sqa_attn_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "sqa_attn_fwd_ex": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "sqa_attn_fwd_cross": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "sqa_attn_fwd_window": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "sqa_attn_fwd_packed": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "sqa_attn_bwd_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "sqa_attn_bwd": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I,
                           _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "sqa_attn_bwd_cross": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I,
                                 _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
+    "sqa_attn_bwd_window": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I,
+                                 _I, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "sqa_attn_bwd_packed": (_I, [_P, _P, _I, _P, _P, _P, _I,
                                  _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "sqa_attn_bwd_static": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I,
@@ -143,6 +146,14 @@ def sqa_attn_fwd_cross(q, k, v, out, out_dtype, lse, B, N_q, N_kv, H_q, H_kv, d_
                                         _stream(stream)), "sqa_attn_fwd_cross")
 
 
+def sqa_attn_fwd_window(q, k, v, out, out_dtype, lse, B, N, H_q, H_kv, d_head, window_left, window_right,
+                        scale, stream=None) -> None:
+    """Sliding-window forward: query t sees keys t - left .. t + right."""
+    _check(library().sqa_attn_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(out_dtype), _ptr(lse),
+                                         B, N, H_q, H_kv, d_head, int(window_left), int(window_right),
+                                         float(scale), _stream(stream)), "sqa_attn_fwd_window")
+
+
 def sqa_attn_fwd_packed(qkv, out, out_dtype, lse, B, N, H_q, H_kv, d_head, causal, scale,
                         stream=None) -> None:
     """Forward on a packed QKV buffer [B, N, H_q + 2*H_kv, d_head]."""
@@ -172,6 +183,16 @@ def sqa_attn_bwd_cross(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype,
                                         B, N_q, N_kv, H_q, H_kv, d_head, float(scale),
                                         _ptr(workspace), int(workspace_bytes), _stream(stream)),
            "sqa_attn_bwd_cross")
+
+
+def sqa_attn_bwd_window(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B, N, H_q, H_kv, d_head,
+                        window_left, window_right, scale, workspace, workspace_bytes, stream=None) -> None:
+    """Gradient of sqa_attn_fwd_window (same window)."""
+    _check(library().sqa_attn_bwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(o_dtype), _ptr(dout),
+                                         _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), int(grad_dtype),
+                                         B, N, H_q, H_kv, d_head, int(window_left), int(window_right),
+                                         float(scale), _ptr(workspace), int(workspace_bytes), _stream(stream)),
+           "sqa_attn_bwd_window")
 
 
 def sqa_attn_bwd_packed(qkv, out, o_dtype, dout, lse, dqkv, grad_dtype, B, N, H_q, H_kv, d_head, causal,

@@ -75,10 +75,12 @@ sqa_status_t check_attn_args(const void* q, const void* k, const void* v, int B,
 }
 
 // Key/value length: any positive length without a mask (cross / memory
-// attention); a causal mask needs as many keys as queries.
-sqa_status_t check_kv_length(int B, int N, int Nkv, int H_kv, int causal) {
+// attention); a causal or windowed mask needs as many keys as queries.
+sqa_status_t check_kv_length(int B, int N, int Nkv, int H_kv, int masked) {
   if (Nkv <= 0) return SQA_ERR_INVALID_ARG;
-  if (causal && Nkv != N) return SQA_ERR_INVALID_ARG;
+  if (masked && Nkv != N) return SQA_ERR_INVALID_ARG;
+  // Band arithmetic (t + win_r + 1 with win_r <= N) stays in 32 bits.
+  if (masked && N > (1 << 30)) return SQA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * Nkv * H_kv > (1ll << 31) - 1) return SQA_ERR_UNSUPPORTED;
   return SQA_OK;
 }
@@ -87,7 +89,10 @@ sqa_status_t check_kv_length(int B, int N, int Nkv, int H_kv, int causal) {
 // the number of elements from one token's row of heads to the next: H * d for
 // the dense layouts, (H_q + 2 H_kv) * d inside a packed QKV buffer.
 struct AttnDesc {
-  int B, N, Nkv, H_q, H_kv, d, causal;
+  int B, N, Nkv, H_q, H_kv, d;
+  int masked;         // band mask: t - win_l <= u <= t + win_r
+  int win_l, win_r;   // clamped to N; causal is (N, 0)
+  int longest_first;  // masked problems: schedule the last token blocks first
   float scale;
   long long ld_q, ld_kv;    // Q; K and V
   long long ld_dq, ld_dkv;  // dQ; dK and dV (backward only)
@@ -101,7 +106,10 @@ AttnDesc dense_desc(int B, int N, int Nkv, int H_q, int H_kv, int d, int causal,
   a.H_q = H_q;
   a.H_kv = H_kv;
   a.d = d;
-  a.causal = causal ? 1 : 0;
+  a.masked = causal ? 1 : 0;
+  a.win_l = N;
+  a.win_r = 0;
+  a.longest_first = a.masked;
   a.scale = scale;
   a.ld_q = a.ld_dq = static_cast<long long>(H_q) * d;
   a.ld_kv = a.ld_dkv = static_cast<long long>(H_kv) * d;
@@ -115,11 +123,22 @@ AttnDesc packed_desc(int B, int N, int H_q, int H_kv, int d, int causal, float s
   return a;
 }
 
+// Sliding window: query t sees keys t - left <= u <= t + right.  Sides of
+// N or more are unbounded, so (>= N, 0) is the causal mask.
+AttnDesc window_desc(int B, int N, int H_q, int H_kv, int d, int left, int right, float scale) {
+  AttnDesc a = dense_desc(B, N, N, H_q, H_kv, d, 1, scale);
+  a.win_l = left < N ? left : N;
+  a.win_r = right < N ? right : N;
+  a.longest_first = a.win_r == 0 && a.win_l == N;
+  return a;
+}
+
 sqa_status_t check_desc(const void* q, const void* k, const void* v, const AttnDesc& a) {
   sqa_status_t s = check_attn_args(q, k, v, a.B, a.N, a.H_q, a.H_kv, a.d, a.scale);
   if (s != SQA_OK) return s;
-  s = check_kv_length(a.B, a.N, a.Nkv, a.H_kv, a.causal);
+  s = check_kv_length(a.B, a.N, a.Nkv, a.H_kv, a.masked);
   if (s != SQA_OK) return s;
+  if (a.win_l < 0 || a.win_r < 0) return SQA_ERR_INVALID_ARG;
   // Token rows are whole 16-byte units (a TMA stride rule) and the element
   // offsets of the last token of the last batch fit in 32-bit row arithmetic.
   const long long lds[4] = {a.ld_q, a.ld_kv, a.ld_dq, a.ld_dkv};
@@ -184,7 +203,10 @@ sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* ou
   p.log2g = log2g;
   p.n_sub = G / g;
   p.n_tblk = (N + 2 * T - 1) / (2 * T);
-  p.causal = a.causal;
+  p.masked = a.masked;
+  p.win_l = a.win_l;
+  p.win_r = a.win_r;
+  p.longest_first = a.longest_first;
   p.out_bf16 = out_bf16;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const long long gy = static_cast<long long>(H_kv) * p.n_sub;
@@ -281,7 +303,10 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
   p.log2g = log2g;
   p.n_sub = G / g;
   p.n_tblk = (N + T - 1) / T;
-  p.causal = a.causal;
+  p.masked = a.masked;
+  p.win_l = a.win_l;
+  p.win_r = a.win_r;
+  p.longest_first = a.longest_first;
   p.scale = a.scale;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.ld_dq = static_cast<int>(a.ld_dq);
@@ -462,6 +487,13 @@ sqa_status_t sqa_attn_fwd_cross(const void* q, const void* k, const void* v, voi
                        stream);
 }
 
+sqa_status_t sqa_attn_fwd_window(const void* q, const void* k, const void* v, void* out, sqa_dtype_t out_dtype,
+                                 float* lse, int B, int N, int H_q, int H_kv, int d_head, int window_left,
+                                 int window_right, float scale, void* stream) {
+  return attn_fwd_impl(q, k, v, out, out_dtype, lse,
+                       window_desc(B, N, H_q, H_kv, d_head, window_left, window_right, scale), stream);
+}
+
 sqa_status_t sqa_attn_fwd_packed(const void* qkv, void* out, sqa_dtype_t out_dtype, float* lse, int B, int N,
                                  int H_q, int H_kv, int d_head, int causal, float scale, void* stream) {
   if (H_q <= 0 || H_kv <= 0 || d_head <= 0 || H_q > (1 << 20) || H_kv > (1 << 20)) return SQA_ERR_INVALID_ARG;
@@ -488,6 +520,16 @@ sqa_status_t sqa_attn_bwd_cross(const void* q, const void* k, const void* v, con
                                 float scale, void* workspace, size_t workspace_bytes, void* stream) {
   return attn_bwd_impl(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype,
                        dense_desc(B, N_q, N_kv, H_q, H_kv, d_head, 0, scale), workspace, workspace_bytes, stream);
+}
+
+sqa_status_t sqa_attn_bwd_window(const void* q, const void* k, const void* v, const void* out, sqa_dtype_t o_dtype,
+                                 const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                                 sqa_dtype_t grad_dtype, int B, int N, int H_q, int H_kv, int d_head,
+                                 int window_left, int window_right, float scale, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  return attn_bwd_impl(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype,
+                       window_desc(B, N, H_q, H_kv, d_head, window_left, window_right, scale), workspace,
+                       workspace_bytes, stream);
 }
 
 sqa_status_t sqa_attn_bwd_packed(const void* qkv, const void* out, sqa_dtype_t o_dtype, const void* dout,

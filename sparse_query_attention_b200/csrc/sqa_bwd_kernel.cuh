@@ -5,6 +5,8 @@
 //   dS   = P o (dO_h V_j^T - D)
 //   dQ_h = scale dS K_j
 //   dK_j = scale sum_{h in group j} dS^T Q_h
+// P is zero outside the visible keys: all keys, or the band
+// t - win_l <= u <= t + win_r (causal, or a sliding window).
 // The training-time gains the pages report ("ReactiveAI/GQA-Ref-Micro" model
 // card, results; "Sparse Query Attention (SQA): ...", abstract: pre-training
 // and fine-tuning) come from these contractions also running over H_q heads
@@ -120,7 +122,9 @@ struct BwdParams {
   int Nkv;                        // key/value tokens (N for self-attention)
   int ld_dq, ld_dkv;              // token strides (elements) of dQ and of dK/dV
   int g, log2g, n_sub, n_tblk;  // packing of the dQ kernel
-  int causal;
+  int masked;                   // band mask active (causal or sliding window)
+  int win_l, win_r;             // band: t - win_l <= u <= t + win_r (both <= N)
+  int longest_first;            // dQ: schedule token blocks from the last one
   float scale;
   float scale_log2;
 };
@@ -182,9 +186,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int j = blockIdx.y;
   const int b = blockIdx.z;
   const int key0 = kt * 128;
-  const int n_qsub = (p.N + 63) / 64;
-  const int qs_begin = p.causal ? (key0 / 64) : 0;
-  const int per_head = n_qsub - qs_begin;
+  // Queries that can see a key of this tile: t in [key0 - win_r,
+  // key0 + 127 + win_l] within [0, N); streamed as 64-token sub-tiles.
+  const int q_lo = p.masked ? max(0, key0 - p.win_r) : 0;
+  const int q_hi = p.masked ? min(p.N, key0 + 128 + p.win_l) : p.N;
+  const int qs_begin = q_lo / 64;
+  const int per_head = max(0, (q_hi + 63) / 64 - qs_begin);
   const int n_steps = p.G * per_head;
 
   if (threadIdx.x == 0) {
@@ -324,10 +331,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float* l2 = reinterpret_cast<const float*>(stat);
       const float* dd = reinterpret_cast<const float*>(stat + 256);
       const int q0 = (qs_begin + s % per_head) * 64;
-      // Query column c (token q0 + c) contributes iff q0 + c < N and, when
-      // causal, q0 + c >= u.  Full tiles skip the per-element test.
-      const int lo = p.causal ? u - q0 : 0;  // first allowed column
-      const int hi = p.N - q0;               // columns [0, hi) are < N
+      // Query column c (token q0 + c) contributes iff q0 + c < N and key u
+      // is inside its band: u - win_r <= q0 + c <= u + win_l.  Full tiles
+      // skip the per-element test.
+      int lo = 0, hi = p.N - q0;  // columns [lo, hi) contribute
+      if (p.masked) {
+        lo = u - p.win_r - q0;
+        hi = min(hi, u + p.win_l - q0 + 1);
+      }
       const bool full = __all_sync(0xffffffffu, lo <= 0 && hi >= 64);
       tmem_wait_ld();
       uint32_t pk[32], dk[32];
@@ -450,14 +461,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = warp_id_uniform();
   const int lane = threadIdx.x & 31;
   const int T = 128 >> p.log2g;
-  const int tblk = p.causal ? (p.n_tblk - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
+  const int tblk = p.longest_first ? (p.n_tblk - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
   const int j = blockIdx.y / p.n_sub;
   const int sub = blockIdx.y % p.n_sub;
   const int b = blockIdx.z;
   const int h0 = j * p.G + sub * p.g;
   const int t0 = tblk * T;
   const int last_tok = min(t0 + T, p.N) - 1;
-  const int n_steps = p.causal ? (last_tok / 64 + 1) : (p.Nkv + 63) / 64;  // 64-key sub-tiles
+  // Keys visible to some row of the tile: [t0 - win_l, last_tok + win_r]
+  // within [0, Nkv), streamed as 64-key sub-tiles from ks_begin.
+  const int k_lo = p.masked ? max(0, t0 - p.win_l) : 0;
+  const int k_hi = p.masked ? min(p.Nkv, last_tok + p.win_r + 1) : p.Nkv;
+  const int ks_begin = k_lo / 64;
+  const int n_steps = max(0, (k_hi + 63) / 64 - ks_begin);
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
@@ -498,8 +514,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         uint8_t* dst = stages + st * C::kStageBytes;
         mbar_arrive_expect_tx(&st_full[st], 2 * KS::kBytes);
         for (int c = 0; c < KS::kChunks; ++c) {
-          tma_load_4d(&tm_k, &st_full[st], dst + c * KS::kChunkBytes, c * KS::kRowElems, j, s * 64, b);
-          tma_load_4d(&tm_v, &st_full[st], dst + KS::kBytes + c * KS::kChunkBytes, c * KS::kRowElems, j, s * 64, b);
+          const int key = (ks_begin + s) * 64;
+          tma_load_4d(&tm_k, &st_full[st], dst + c * KS::kChunkBytes, c * KS::kRowElems, j, key, b);
+          tma_load_4d(&tm_v, &st_full[st], dst + KS::kBytes + c * KS::kChunkBytes, c * KS::kRowElems, j, key, b);
         }
       }
       mbar_drain(&q_full, 0);
@@ -584,10 +601,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tmem_ld32(lane_base + C::col_s(buf) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_ld32(lane_base + C::col_dp(buf), *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
       tmem_ld32(lane_base + C::col_dp(buf) + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
-      const int kbase = s * 64;
-      int hi = p.Nkv - kbase;                      // keys [0, hi) exist
-      if (p.causal) hi = min(hi, tok - kbase + 1);  // keys <= tok
-      const bool full = __all_sync(0xffffffffu, hi >= 64);
+      const int kbase = (ks_begin + s) * 64;
+      int lo = 0, hi = p.Nkv - kbase;  // keys [lo, hi) of the sub-tile are visible
+      if (p.masked) {
+        lo = tok - p.win_l - kbase;
+        hi = min(hi, tok + p.win_r - kbase + 1);
+      }
+      const bool full = __all_sync(0xffffffffu, lo <= 0 && hi >= 64);
       tmem_wait_ld();
       uint32_t dk[32];
       // dS = 2^(s sl2 - L2) (dP - D) with the row's -L2 and -D (nl2, ndd),
@@ -608,8 +628,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const uint64_t t = f2_add(f2_pack(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])), ndd2);
           f2_unpack(f2_mul(f2_pack(p0, p1), t), d0, d1);
           if constexpr (decltype(masked)::value) {
-            d0 = c < hi ? d0 : 0.f;
-            d1 = c + 1 < hi ? d1 : 0.f;
+            d0 = (c >= lo && c < hi) ? d0 : 0.f;
+            d1 = (c + 1 >= lo && c + 1 < hi) ? d1 : 0.f;
           }
           dk[c2] = pack_bf16x2(d0, d1);
         }

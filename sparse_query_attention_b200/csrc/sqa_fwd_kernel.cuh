@@ -4,7 +4,9 @@
 // G = H_q / H_kv):
 //   O[b,t,h,:] = sum_u softmax_u(scale * <Q[b,t,h,:], K[b,u,j,:]>) V[b,u,j,:]
 //   LSE[b,h,t] = log sum_u exp(scale * <Q[b,t,h,:], K[b,u,j,:]>)
-// with u <= t when causal.  Only H_q query heads exist, so the two
+// over the keys u visible to query t: all of them, or the band
+// t - win_l <= u <= t + win_r (causal: win_l >= N, win_r = 0; a sliding
+// window otherwise).  Only H_q query heads exist, so the two
 // contractions cost 2 * B * H_q * P_c * d FLOPs each: the query-head
 // reduction of "Sparse Query Attention (SQA): A Computationally Efficient
 // Attention Mechanism with Query Heads Reduction" (abstract), built on the
@@ -60,7 +62,9 @@ struct FwdParams {
   int Nkv;         // key/value tokens (N for self-attention; causal needs Nkv == N)
   int n_sub;       // G / g head sub-groups per KV head
   int n_tblk;      // token blocks of 2 * (128 / g) tokens
-  int causal;
+  int masked;      // band mask active (causal or sliding window)
+  int win_l, win_r;  // band: t - win_l <= u <= t + win_r (both <= N)
+  int longest_first;  // schedule token blocks from the last one
   int out_bf16;
   float scale_log2;  // scale * log2(e)
 };
@@ -98,24 +102,29 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   // ---- work unit -----------------------------------------------------------
   const int T = 128 >> p.log2g;  // tokens per tile
-  const int tblk = p.causal ? (p.n_tblk - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
+  const int tblk = p.longest_first ? (p.n_tblk - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
   const int j = blockIdx.y / p.n_sub;
   const int sub = blockIdx.y % p.n_sub;
   const int b = blockIdx.z;
   const int h0 = j * p.G + sub * p.g;
   const int t0 = tblk * 2 * T;  // tile 0 tokens [t0, t0+T), tile 1 [t0+T, t0+2T)
-  const int n_kv_all = (p.Nkv + 127) / 128;
-  int n_kv[2];
+  // KV tiles [kv_lo[t], kv_hi[t]) hold every key a row of query tile t can
+  // see; the CTA streams the union [kv_begin, kv_begin + n_steps).  Tile 0
+  // always has tokens (t0 < N); a tile 1 entirely past N gets an empty range,
+  // runs its steps fully masked so its barriers stay in lock-step, and
+  // stores nothing.
+  int kv_lo[2], kv_hi[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    const int last_tok = min(t0 + (t + 1) * T, p.N) - 1;
-    n_kv[t] = p.causal ? (last_tok < 0 ? 0 : last_tok / 128 + 1) : n_kv_all;
+    const int tmin = t0 + t * T, tmax = min(t0 + (t + 1) * T, p.N) - 1;
+    const int lo = p.masked ? max(0, tmin - p.win_l) : 0;
+    const int hi = p.masked ? min(p.Nkv, tmax + p.win_r + 1) : p.Nkv;
+    kv_lo[t] = lo / 128;
+    kv_hi[t] = (hi + 127) / 128;
   }
-  // A tile entirely past N still runs one (masked) step so its barriers stay
-  // in lock-step; its rows are never stored.
-  n_kv[0] = max(n_kv[0], 1);
-  n_kv[1] = max(n_kv[1], 1);
-  const int n_steps = max(n_kv[0], n_kv[1]);
+  const int kv_begin = kv_lo[0];
+  if (t0 + T >= p.N) kv_lo[1] = kv_hi[1] = kv_begin;  // tile 1 holds no token
+  const int n_steps = max(1, max(kv_hi[0], kv_hi[1]) - kv_begin);
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
@@ -174,7 +183,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           uint8_t* dst = ring + s * C::kTileBytes;
           const CUtensorMap* m = kv == 0 ? &tm_k : &tm_v;
           for (int c = 0; c < C::kChunks; ++c)
-            tma_load_4d(m, &slot_full[s], dst + c * C::kChunkBytes, c * C::kRowElems, j, i * 128, b);
+            tma_load_4d(m, &slot_full[s], dst + c * C::kChunkBytes, c * C::kRowElems, j, (kv_begin + i) * 128, b);
         }
       }
       // Teardown: nothing may still be landing in shared memory at exit.
@@ -277,6 +286,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t o_addr = lane_base + (t == 0 ? C::kColO0 : C::kColO1);
     const float sl2 = p.scale_log2;
     const int tile_tok_min = t0 + t * T;
+    const int tile_tok_max = min(tile_tok_min + T, p.N) - 1;
     const int my_steps = n_steps;  // both tiles step in lock-step with the MMA warp
 
     float m_used = -INFINITY;  // running max in log2 units (of scaled scores)
@@ -297,19 +307,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       float s[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
-      // Masking: keys past N, and keys after the query token when causal.
-      // Unmasked tiles (the common case) keep raw scores: the row max is
-      // taken on them and the scale is folded into the exponent's FFMA.
-      // Masked tiles are scaled first and get -inf where masked.
-      const int key0 = i * 128;
-      const bool need_mask = (key0 + 128 > p.Nkv) || (p.causal && key0 + 127 > tile_tok_min) || i >= n_kv[t];
+      // Masking: keys past Nkv, keys outside the band, and whole tiles
+      // outside this query tile's range.  Unmasked tiles (the common case)
+      // keep raw scores: the row max is taken on them and the scale is
+      // folded into the exponent's FFMA.  Masked tiles are scaled first and
+      // get -inf where masked.
+      const int kt = kv_begin + i;
+      const int key0 = kt * 128;
+      const bool outside = kt < kv_lo[t] || kt >= kv_hi[t];
+      const bool need_mask = (key0 + 128 > p.Nkv) || outside ||
+                             (p.masked && (key0 + 127 > tile_tok_min + p.win_r || key0 < tile_tok_max - p.win_l));
       float mult = sl2;  // exponent argument = s * mult - m
       if (need_mask) {
-        int lim = p.Nkv - key0;                                 // keys [0, lim) exist
-        if (p.causal) lim = min(lim, tok - key0 + 1);           // keys <= tok
-        if (i >= n_kv[t]) lim = 0;
+        int lo = 0, lim = p.Nkv - key0;  // columns [lo, lim) are visible
+        if (p.masked) {
+          lo = tok - p.win_l - key0;
+          lim = min(lim, tok + p.win_r - key0 + 1);
+        }
+        if (outside) lim = 0;
 #pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = c < lim ? s[c] * sl2 : -INFINITY;
+        for (int c = 0; c < 128; ++c) s[c] = (c >= lo && c < lim) ? s[c] * sl2 : -INFINITY;
         mult = 1.f;
       }
       // Row max (row min for a negative scale on raw scores): eight

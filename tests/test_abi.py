@@ -25,6 +25,7 @@ def test_header_declares_expected_entry_points():
     names = _declared_symbols()
     for n in ("sqa_attn_fwd", "sqa_attn_fwd_ex", "sqa_attn_bwd", "sqa_attn_bwd_workspace_size",
               "sqa_attn_fwd_cross", "sqa_attn_bwd_cross", "sqa_attn_fwd_packed", "sqa_attn_bwd_packed",
+              "sqa_attn_fwd_window", "sqa_attn_bwd_window",
               "sqa_proj", "sqa_device_status", "sqa_status_string", "sqa_version"):
         assert n in names
 
@@ -107,6 +108,20 @@ def test_cross_rejects_invalid_lengths():
     # The workspace holds per-query-row values: sized for N_q, not N_kv.
     assert lib.sqa_attn_bwd_cross(FAKE, FAKE, FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1, 4096, 8, 4, 2, 32,
                                   0.1, FAKE, ws, None) == sqa.SQA_ERR_INVALID_ARG
+
+
+def test_window_rejects_invalid_arguments():
+    lib = sqa.library()
+    for left, right in ((-1, 0), (0, -1), (-5, -5)):
+        assert lib.sqa_attn_fwd_window(FAKE, FAKE, FAKE, FAKE, 0, None, 1, 8, 4, 2, 32, left, right, 0.1,
+                                       None) == sqa.SQA_ERR_INVALID_ARG
+    assert lib.sqa_attn_fwd_window(FAKE, FAKE, FAKE, FAKE, 0, None, 1, 0, 4, 2, 32, 3, 0, 0.1,
+                                   None) == sqa.SQA_ERR_INVALID_ARG
+    ws = sqa.sqa_attn_bwd_workspace_size(1, 8, 4, 2, 32)
+    assert lib.sqa_attn_bwd_window(FAKE, FAKE, FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1, 8, 4, 2, 32,
+                                   -1, 0, 0.1, FAKE, ws, None) == sqa.SQA_ERR_INVALID_ARG
+    assert lib.sqa_attn_bwd_window(FAKE, FAKE, FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1, 8, 4, 2, 32,
+                                   2, 2, 0.1, FAKE, ws - 4, None) == sqa.SQA_ERR_INVALID_ARG
 
 
 def test_packed_rejects_invalid_arguments():
