@@ -10,6 +10,7 @@ does.
 from .sqa_oracle import (  # noqa: F401
     attention_forward,
     attention_backward,
+    attention_decode,
     projection,
     projection_backward,
     sqa_layer_backward,

@@ -179,6 +179,46 @@ def attention_backward(q, k, v, do, causal: bool, scale: float, window=None):
     return dq, dk, dv
 
 
+def attention_decode(q, k_cache, v_cache, cache_lens, scale: float):
+    """Decoding against a key/value cache: autoregressive inference, whose
+    latency the abstract of "Sparse Query Attention (SQA): ..." describes as
+    bound by memory bandwidth (the regime MQA/GQA address by sharing K/V),
+    unlike the compute-bound training and full-sequence work SQA targets.
+
+    q: [B, n_new, H_q, d], the queries of the last n_new tokens of each
+    sequence; k_cache, v_cache: [B, L_max, H_kv, d], of which the first
+    cache_lens[b] tokens of sequence b are valid (the new tokens' keys and
+    values included, so n_new <= cache_lens[b] <= L_max); the rest is never
+    read.  Token i of sequence b sits at position p = cache_lens[b] - n_new + i
+    and sees keys 0..p (the causal rule).
+    Returns o [B, n_new, H_q, d] and lse [B, H_q, n_new].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    B, n_new, H_q, d = q.shape
+    H_kv = k_cache.shape[2]
+    G = _check_heads(H_q, H_kv)
+    L_max = k_cache.shape[1]
+    o = np.empty((B, n_new, H_q, d), dtype=np.float64)
+    lse = np.empty((B, H_q, n_new), dtype=np.float64)
+    for b in range(B):
+        L = int(cache_lens[b])
+        if not n_new <= L <= L_max:
+            raise ValueError(f"cache length {L} outside [{n_new}, {L_max}]")
+        k = np.asarray(k_cache[b, :L], dtype=np.float64)
+        v = np.asarray(v_cache[b, :L], dtype=np.float64)
+        pos = L - n_new + np.arange(n_new)
+        for h in range(H_q):
+            j = h // G
+            s = scale * (q[b, :, h, :] @ k[:, j, :].T)
+            s[np.arange(L)[None, :] > pos[:, None]] = -np.inf
+            m = s.max(axis=1, keepdims=True)
+            w = np.exp(s - m)
+            l = w.sum(axis=1)
+            o[b, :, h, :] = (w @ v[:, j, :]) / l[:, None]
+            lse[b, h, :] = m[:, 0] + np.log(l)
+    return o, lse
+
+
 def projection(x, w, bias=None):
     """y = x w^T (+ bias): x [M, K], w [Nout, K] in nn.Linear layout."""
     y = np.asarray(x, dtype=np.float64) @ np.asarray(w, dtype=np.float64).T

@@ -21,8 +21,8 @@ import pytest
 import torch
 import torch.nn.functional as F
 
-from oracle import (attention_backward, attention_forward, projection, projection_backward, sqa_layer_backward,
-                    sqa_layer_forward)
+from oracle import (attention_backward, attention_decode, attention_forward, projection, projection_backward,
+                    sqa_layer_backward, sqa_layer_forward)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "closed_form_cases.json")
 
@@ -554,3 +554,68 @@ def test_window_rejects_bad_arguments():
         attention_forward(z, z, z, False, 1.0, window=(-1, 0))
     with pytest.raises(ValueError):
         attention_forward(z, np.zeros((1, 5, 1, 2)), np.zeros((1, 5, 1, 2)), False, 1.0, window=(2, 2))
+
+
+# ---------------------------------------------------------------------------
+# KV-cache decode
+# ---------------------------------------------------------------------------
+def _decode_case(rng, B, n_new, H_q, H_kv, d, lens, L_max):
+    q = _rand((B, n_new, H_q, d), rng)
+    kc = _rand((B, L_max, H_kv, d), rng)
+    vc = _rand((B, L_max, H_kv, d), rng)
+    return q, kc, vc, np.asarray(lens)
+
+
+@pytest.mark.parametrize("n_new,heads", [(1, (4, 2)), (3, (4, 4)), (2, (8, 1))])
+def test_decode_matches_sdpa_last_rows(n_new, heads):
+    """Decoding n_new tokens equals the last n_new rows of causal attention
+    over the sequence's first len_b tokens (torch SDPA, fp64), per sequence,
+    with ragged lengths."""
+    H_q, H_kv = heads
+    rng = np.random.default_rng(40 + n_new)
+    B, d, L_max = 3, 8, 23
+    lens = [23, 5, 14][:B]
+    q, kc, vc, lens = _decode_case(rng, B, n_new, H_q, H_kv, d, lens, L_max)
+    scale = 1 / math.sqrt(d)
+    o, lse = attention_decode(q, kc, vc, lens, scale)
+    for b in range(B):
+        L = lens[b]
+        qf = _rand((L, H_q, d), rng)      # earlier rows: arbitrary, they only fill the sequence
+        qf[L - n_new:] = q[b]
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).permute(1, 0, 2)[None]
+        ref = F.scaled_dot_product_attention(t(qf), t(kc[b, :L]), t(vc[b, :L]), is_causal=True, scale=scale,
+                                             enable_gqa=H_q != H_kv)
+        np.testing.assert_allclose(o[b], ref[0].permute(1, 0, 2).numpy()[L - n_new:], atol=1e-12)
+
+
+def test_decode_brute_force_and_unused_cache():
+    """fsum brute force with explicit key lists; cache entries past len_b
+    (here NaN) are never read."""
+    rng = np.random.default_rng(5)
+    B, n_new, H_q, H_kv, d, L_max = 2, 2, 4, 2, 3, 9
+    q, kc, vc, lens = _decode_case(rng, B, n_new, H_q, H_kv, d, [9, 4], L_max)
+    kc[1, 4:] = np.nan
+    vc[1, 4:] = np.nan
+    o, lse = attention_decode(q, kc, vc, lens, 0.6)
+    for b in range(B):
+        L = int(lens[b])
+        for h in range(H_q):
+            j = h // 2
+            for i in range(n_new):
+                keys = range(L - n_new + i + 1)
+                e = [math.exp(0.6 * math.fsum(q[b, i, h, c] * kc[b, u, j, c] for c in range(d))) for u in keys]
+                z = math.fsum(e)
+                for c in range(d):
+                    assert abs(o[b, i, h, c] - math.fsum(e[u] * vc[b, u, j, c] for u in keys) / z) < 1e-12
+                assert abs(lse[b, h, i] - math.log(z)) < 1e-12
+
+
+def test_decode_single_key_and_rejects_bad_lengths():
+    rng = np.random.default_rng(6)
+    q, kc, vc, lens = _decode_case(rng, 1, 1, 2, 1, 4, [1], 5)
+    o, lse = attention_decode(q, kc, vc, lens, 0.5)
+    np.testing.assert_allclose(o[0, 0], np.repeat(vc[0, 0], 2, axis=0), atol=1e-15)
+    np.testing.assert_allclose(lse[0, :, 0], 0.5 * (q[0, 0] @ kc[0, 0, 0]), atol=1e-14)
+    for bad in ([0], [6]):
+        with pytest.raises(ValueError):
+            attention_decode(q, kc, vc, np.asarray(bad), 0.5)
