@@ -325,6 +325,62 @@ def time_windowed(sqa, torch, stream, dev, reps=3):
     return {"config": {"B": 1, "N": N, "d_head": d}, "windows": res}
 
 
+DECODE = {"B": 16, "L": 32768, "n_new": 1, "d_head": 128}
+DECODE_VARIANTS = {"MHA": (16, 16), "GQA": (16, 4), "SQA": (8, 4), "xSQA": (4, 4), "xSMQA": (4, 1)}
+
+
+def load_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f).get("hbm_gbs", 6650.0), "measured"
+    return 6650.0, "fallback"
+
+
+def time_decode(sqa, torch, stream, dev, reps=10):
+    """One decode step (n_new = 1) for B = 16 sequences with 32768 cached
+    tokens, d = 128, per head-count variant.  HBM-bound: algorithmic bytes
+    are the K and V cache (2 * B * L * H_kv * d bf16) plus Q and O; the cache
+    is larger than L2 at every variant but xSMQA (128 MiB), so no flush is
+    added.  Reported against the measured copy bandwidth."""
+    c = DECODE
+    B, L, n_new, d = c["B"], c["L"], c["n_new"], c["d_head"]
+    peak, kind = load_hbm_peak()
+    res = {}
+    for name, (hq, hkv) in DECODE_VARIANTS.items():
+        g = torch.Generator(device=dev)
+        g.manual_seed(5)
+        q = torch.randn((B, n_new, hq, d), generator=g, device=dev).to(torch.bfloat16)
+        kc = torch.randn((B, L, hkv, d), generator=g, device=dev).to(torch.bfloat16)
+        vc = torch.randn((B, L, hkv, d), generator=g, device=dev).to(torch.bfloat16)
+        lens = torch.full((B,), L, dtype=torch.int32, device=dev)
+        out = torch.empty((B, n_new, hq, d), dtype=torch.bfloat16, device=dev)
+        wsb = sqa.sqa_attn_decode_workspace_size(B, n_new, hq, hkv, d, L)
+        ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=dev)
+
+        def step():
+            sqa.sqa_attn_decode(q, kc, vc, lens, out, sqa.SQA_DT_BF16, None, B, n_new, hq, hkv, d, L,
+                                1 / math.sqrt(d), ws if wsb else None, wsb, stream=stream)
+
+        for _ in range(3):
+            step()
+        times = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            step()
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        ms = statistics.median(times)
+        nbytes = 2 * B * L * hkv * d * 2 + 2 * B * n_new * hq * d * 2
+        res[name] = {"H_q": hq, "H_kv": hkv, "ms": ms, "gbs": nbytes / ms / 1e6, "frac_hbm": nbytes / ms / 1e6 / peak,
+                     "tokens_per_s": B * n_new / (ms / 1e3)}
+        del q, kc, vc, out, ws
+    sqa.sqa_device_status(stream)
+    return {"config": dict(c), "hbm_peak_gbs": peak, "hbm_peak_source": f"{kind} copy", "variants": res}
+
+
 LAYER = {"B": 16, "N": 1024, "d_model": 256, "d_head": 16, "causal": True}
 LAYER_VARIANTS = {"MHA": (16, 16), "GQA": (16, 4), "SQA": (8, 4), "sSQA": (8, 8), "xSQA": (4, 4), "xSMQA": (4, 1)}
 
@@ -571,6 +627,7 @@ def run_sqa(args):
     layer = time_decoder_layer(sqa, torch, stream, flush, dev)
     long_seq = time_long_sequences(sqa, torch, stream, dev)
     windowed = time_windowed(sqa, torch, stream, dev)
+    decode = time_decode(sqa, torch, stream, dev)
 
     peak, peak_kind = load_peaks()
     achieved = flops_step / (statistics.mean(per_launch_ms) / 1e3) / 1e12
@@ -593,6 +650,7 @@ def run_sqa(args):
         "decoder_layer": layer,
         "long_sequences": long_seq,
         "windowed": windowed,
+        "decode": decode,
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

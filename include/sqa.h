@@ -171,6 +171,37 @@ sqa_status_t sqa_attn_bwd_window(const void* q, const void* k, const void* v,
                                  void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * sqa_attn_decode - decoding against a key/value cache.  Autoregressive
+ * inference is the memory-bound regime ("Sparse Query Attention (SQA): ...",
+ * abstract: its latency is bound by memory bandwidth, which MQA/GQA address
+ * by sharing K/V): each step streams the cache once, so SQA's fewer query
+ * heads cut arithmetic but not bytes; the kernel is built to stream the cache
+ * at HBM speed.
+ * Inputs : q [B, n_new, H_q, d_head] bf16, the queries of the last n_new
+ *          tokens of each sequence;
+ *          k_cache, v_cache [B, L_max, H_kv, d_head] bf16, of which the first
+ *          cache_lens[b] tokens of sequence b are valid, the new tokens' own
+ *          keys/values included; entries past cache_lens[b] are never read;
+ *          cache_lens: DEVICE int32 [B], n_new <= cache_lens[b] <= L_max.
+ * Outputs: out [B, n_new, H_q, d_head] (out_dtype), lse [B, H_q, n_new] fp32
+ *          (natural log) or NULL.  Token i of sequence b sits at position
+ *          cache_lens[b] - n_new + i and sees keys 0 .. that position.
+ * workspace: sqa_attn_decode_workspace_size() bytes (0 when the cache is
+ *          processed as one chunk per sequence; workspace may then be NULL).
+ * Requirements: g * n_new <= 128 where g is the largest power of two dividing
+ * H_q / H_kv (else SQA_ERR_UNSUPPORTED); other rules as sqa_attn_fwd.  A
+ * cache length outside [n_new, L_max] cannot be checked on the host: the
+ * kernel clamps it into range and sqa_device_status() then reports
+ * SQA_ERR_INVALID_ARG.
+ */
+size_t sqa_attn_decode_workspace_size(int B, int n_new, int H_q, int H_kv, int d_head, int L_max);
+
+sqa_status_t sqa_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                             const int* cache_lens, void* out, sqa_dtype_t out_dtype, float* lse,
+                             int B, int n_new, int H_q, int H_kv, int d_head, int L_max,
+                             float scale, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * sqa_attn_fwd_packed - the forward on a packed QKV buffer, the output of one
  * fused input projection with the concatenated weight [Wq; Wk; Wv]
  * ((H_q + 2 H_kv) * d_head rows): qkv [B, N, H_q + 2 H_kv, d_head] bf16,
@@ -269,8 +300,9 @@ sqa_status_t sqa_gemm(const void* a, sqa_layout_t a_layout, const void* b, sqa_l
 /*
  * sqa_device_status - synchronises `stream`, then returns SQA_ERR_TIMEOUT if
  * any kernel of this library on the current device gave up a bounded wait
- * since the last call (and clears the record), SQA_ERR_CUDA if the stream
- * reports an error, else SQA_OK.
+ * since the last call, else SQA_ERR_INVALID_ARG if sqa_attn_decode met a
+ * cache length outside [n_new, L_max] (and clears the record either way),
+ * SQA_ERR_CUDA if the stream reports an error, else SQA_OK.
  */
 sqa_status_t sqa_device_status(void* stream);
 

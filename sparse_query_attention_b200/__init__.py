@@ -36,6 +36,8 @@ SIGNATURES = {
     "sqa_attn_fwd_ex": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "sqa_attn_fwd_cross": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "sqa_attn_fwd_window": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "sqa_attn_decode_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "sqa_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "sqa_attn_fwd_packed": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "sqa_attn_bwd_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "sqa_attn_bwd": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I,
@@ -152,6 +154,19 @@ def sqa_attn_fwd_window(q, k, v, out, out_dtype, lse, B, N, H_q, H_kv, d_head, w
     _check(library().sqa_attn_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(out_dtype), _ptr(lse),
                                          B, N, H_q, H_kv, d_head, int(window_left), int(window_right),
                                          float(scale), _stream(stream)), "sqa_attn_fwd_window")
+
+
+def sqa_attn_decode_workspace_size(B, n_new, H_q, H_kv, d_head, L_max) -> int:
+    return int(library().sqa_attn_decode_workspace_size(B, n_new, H_q, H_kv, d_head, L_max))
+
+
+def sqa_attn_decode(q, k_cache, v_cache, cache_lens, out, out_dtype, lse, B, n_new, H_q, H_kv, d_head, L_max,
+                    scale, workspace, workspace_bytes, stream=None) -> None:
+    """Decode n_new tokens per sequence against a KV cache; cache_lens is a
+    device int32 tensor [B]."""
+    _check(library().sqa_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_lens), _ptr(out),
+                                     int(out_dtype), _ptr(lse), B, n_new, H_q, H_kv, d_head, L_max, float(scale),
+                                     _ptr(workspace), int(workspace_bytes), _stream(stream)), "sqa_attn_decode")
 
 
 def sqa_attn_fwd_packed(qkv, out, out_dtype, lse, B, N, H_q, H_kv, d_head, causal, scale,

@@ -3,6 +3,7 @@
 // the device status word and every kernel live in the same module.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -10,6 +11,7 @@
 
 #include "sqa.h"
 #include "sqa_bwd_kernel.cuh"
+#include "sqa_decode_kernel.cuh"
 #include "sqa_fwd_kernel.cuh"
 #include "sqa_proj_kernel.cuh"
 #include "sqa_ptx.cuh"
@@ -456,6 +458,123 @@ sqa_status_t gemm_impl(const void* a, bool a_mn, const void* b, bool b_mn, const
             : launch_gemm_layouts<false, true, false>(ma, mb, bn, bias, c, M, N, K, accumulate, st);
 }
 
+// ---------------------------------------------------------------------------
+// KV-cache decode
+// ---------------------------------------------------------------------------
+// Chunking of the cache: at least two waves of two CTAs per SM over the
+// (batch, key/value head, head sub-group) units, chunks of at least 256
+// keys and a multiple of the 64-key step; among split counts up to four
+// times that minimum, the smallest whose last wave is at least 95 % full
+// (else the fullest).  Depends only on the shape, so the workspace size is
+// known before the lengths are.
+constexpr int kNumSMs = 148;
+constexpr int kDecodeSlots = 2 * kNumSMs;  // CTAs resident at once
+
+struct DecodePlan {
+  int g, log2g, n_sub, chunk, n_split;
+};
+
+DecodePlan decode_plan(int B, int H_q, int H_kv, int L_max) {
+  DecodePlan pl;
+  const int G = H_q / H_kv;
+  pl.g = head_pack(G);
+  pl.log2g = 0;
+  while ((1 << pl.log2g) < pl.g) ++pl.log2g;
+  pl.n_sub = G / pl.g;
+  const long long units = static_cast<long long>(B) * H_kv * pl.n_sub;
+  const long long max_split = (L_max + 255) / 256 > 0 ? (L_max + 255) / 256 : 1;
+  const long long n_min = std::min(max_split, std::max(1LL, (2LL * kDecodeSlots + units - 1) / units));
+  const long long n_max = std::min(max_split, 4 * n_min);
+  long long n = n_min;
+  double best = -1.0;
+  for (long long c = n_min; c <= n_max; ++c) {
+    const long long ctas = units * c;
+    const double fill = static_cast<double>(ctas) / (((ctas + kDecodeSlots - 1) / kDecodeSlots) * kDecodeSlots);
+    if (fill >= 0.95) {
+      n = c;
+      break;
+    }
+    if (fill > best) {
+      best = fill;
+      n = c;
+    }
+  }
+  const long long per = (L_max + n - 1) / n;
+  pl.chunk = static_cast<int>((per + 63) / 64 * 64);
+  pl.n_split = static_cast<int>((L_max + pl.chunk - 1) / pl.chunk);
+  return pl;
+}
+
+size_t decode_part_l_bytes(int n_split, int B, int n_new, int H_q) {
+  const size_t n = static_cast<size_t>(n_split) * B * n_new * H_q * sizeof(float);
+  return (n + 255) & ~size_t(255);
+}
+
+size_t decode_workspace_bytes(int B, int n_new, int H_q, int H_kv, int d, int L_max) {
+  const DecodePlan pl = decode_plan(B, H_q, H_kv, L_max);
+  if (pl.n_split <= 1) return 0;
+  return decode_part_l_bytes(pl.n_split, B, n_new, H_q) +
+         static_cast<size_t>(pl.n_split) * B * n_new * H_q * d * sizeof(float);
+}
+
+template <int D>
+sqa_status_t launch_decode(const void* q, const void* kc, const void* vc, const int* lens, void* out, int out_bf16,
+                           float* lse, int B, int n_new, int H_q, int H_kv, int L_max, float scale, void* ws,
+                           cudaStream_t st) {
+  using C = sqa::DecCfg<D>;
+  const DecodePlan pl = decode_plan(B, H_q, H_kv, L_max);
+  if (pl.g * n_new > 128) return SQA_ERR_UNSUPPORTED;  // one 128-row query tile per CTA
+  CUtensorMap mq, mk, mv;
+  const CUtensorMapSwizzle swz = tma_swizzle_for_row_bytes(C::kRowBytes);
+  {
+    const uint64_t dims[4] = {uint64_t(D), uint64_t(H_q), uint64_t(n_new), uint64_t(B)};
+    const uint64_t strides[3] = {uint64_t(D) * 2, uint64_t(H_q) * D * 2, uint64_t(n_new) * H_q * D * 2};
+    const uint32_t box[4] = {uint32_t(C::kRowElems), uint32_t(pl.g), uint32_t(n_new), 1};
+    if (!make_map_bf16(&mq, q, 4, dims, strides, box, swz)) return SQA_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[4] = {uint64_t(D), uint64_t(H_kv), uint64_t(L_max), uint64_t(B)};
+    const uint64_t strides[3] = {uint64_t(D) * 2, uint64_t(H_kv) * D * 2, uint64_t(L_max) * H_kv * D * 2};
+    const uint32_t box[4] = {uint32_t(C::kRowElems), 1, uint32_t(C::kBK), 1};
+    if (!make_map_bf16(&mk, kc, 4, dims, strides, box, swz)) return SQA_ERR_CUDA;
+    if (!make_map_bf16(&mv, vc, 4, dims, strides, box, swz)) return SQA_ERR_CUDA;
+  }
+  sqa::DecParams p;
+  p.out = out;
+  p.lse = lse;
+  p.part_l = pl.n_split > 1 ? static_cast<float*>(ws) : nullptr;
+  p.part_o = pl.n_split > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                                       decode_part_l_bytes(pl.n_split, B, n_new, H_q))
+                            : nullptr;
+  p.cache_lens = lens;
+  p.B = B;
+  p.n_new = n_new;
+  p.H_q = H_q;
+  p.H_kv = H_kv;
+  p.G = H_q / H_kv;
+  p.g = pl.g;
+  p.log2g = pl.log2g;
+  p.n_sub = pl.n_sub;
+  p.L_max = L_max;
+  p.chunk = pl.chunk;
+  p.n_split = pl.n_split;
+  p.out_bf16 = out_bf16;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const long long gy = static_cast<long long>(H_kv) * pl.n_sub;
+  if (gy > 65535 || B > 65535) return SQA_ERR_UNSUPPORTED;
+  auto kern = sqa::sqa_decode_kernel<D>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+    return SQA_ERR_CUDA;
+  dim3 grid(pl.n_split, static_cast<unsigned>(gy), B);
+  kern<<<grid, sqa::kDecThreads, C::kSmemBytes, st>>>(mq, mk, mv, p);
+  if (cudaGetLastError() != cudaSuccess) return SQA_ERR_CUDA;
+  if (pl.n_split > 1) {
+    const size_t rows = static_cast<size_t>(B) * n_new * H_q;
+    sqa::decode_combine_kernel<D><<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(p);
+  }
+  return launch_status();
+}
+
 // Byte offset of head `h` within one token row of d-element heads.
 inline const void* head_ptr(const void* base, int h, int d, size_t elem) {
   return base ? static_cast<const uint8_t*>(base) + static_cast<size_t>(h) * d * elem : nullptr;
@@ -492,6 +611,45 @@ sqa_status_t sqa_attn_fwd_window(const void* q, const void* k, const void* v, vo
                                  int window_right, float scale, void* stream) {
   return attn_fwd_impl(q, k, v, out, out_dtype, lse,
                        window_desc(B, N, H_q, H_kv, d_head, window_left, window_right, scale), stream);
+}
+
+size_t sqa_attn_decode_workspace_size(int B, int n_new, int H_q, int H_kv, int d_head, int L_max) {
+  if (B <= 0 || n_new <= 0 || H_q <= 0 || H_kv <= 0 || H_kv > H_q || H_q % H_kv != 0 || d_head <= 0 ||
+      L_max < n_new)
+    return 0;
+  return decode_workspace_bytes(B, n_new, H_q, H_kv, d_head, L_max);
+}
+
+sqa_status_t sqa_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int* cache_lens,
+                             void* out, sqa_dtype_t out_dtype, float* lse, int B, int n_new, int H_q, int H_kv,
+                             int d_head, int L_max, float scale, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  sqa_status_t s = check_attn_args(q, k_cache, v_cache, B, n_new, H_q, H_kv, d_head, scale);
+  if (s != SQA_OK) return s;
+  if (!cache_lens || !out || L_max < n_new) return SQA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cache_lens) & 3u) != 0 || !aligned16(out) || (lse && !aligned16(lse)))
+    return SQA_ERR_INVALID_ARG;
+  if (out_dtype != SQA_DT_F32 && out_dtype != SQA_DT_BF16) return SQA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * L_max * H_kv > (1ll << 31) - 1) return SQA_ERR_UNSUPPORTED;
+  const size_t need = decode_workspace_bytes(B, n_new, H_q, H_kv, d_head, L_max);
+  if (need > 0 && (workspace == nullptr || !aligned16(workspace) || workspace_bytes < need))
+    return SQA_ERR_INVALID_ARG;
+  const int ob = out_dtype == SQA_DT_BF16;
+  cudaStream_t st = as_stream(stream);
+  switch (d_head) {
+    case 16:
+      return launch_decode<16>(q, k_cache, v_cache, cache_lens, out, ob, lse, B, n_new, H_q, H_kv, L_max, scale,
+                               workspace, st);
+    case 32:
+      return launch_decode<32>(q, k_cache, v_cache, cache_lens, out, ob, lse, B, n_new, H_q, H_kv, L_max, scale,
+                               workspace, st);
+    case 64:
+      return launch_decode<64>(q, k_cache, v_cache, cache_lens, out, ob, lse, B, n_new, H_q, H_kv, L_max, scale,
+                               workspace, st);
+    default:
+      return launch_decode<128>(q, k_cache, v_cache, cache_lens, out, ob, lse, B, n_new, H_q, H_kv, L_max, scale,
+                                workspace, st);
+  }
 }
 
 sqa_status_t sqa_attn_fwd_packed(const void* qkv, void* out, sqa_dtype_t out_dtype, float* lse, int B, int N,
@@ -611,7 +769,8 @@ sqa_status_t sqa_device_status(void* stream) {
   if (word != 0) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(sqa::g_status_word, &zero, sizeof(zero)) != cudaSuccess) return SQA_ERR_CUDA;
-    return SQA_ERR_TIMEOUT;
+    // A timed-out wait outranks a clamped decode length.
+    return (word & sqa::kStatusTimeout) ? SQA_ERR_TIMEOUT : SQA_ERR_INVALID_ARG;
   }
   return SQA_OK;
 }

@@ -25,7 +25,7 @@ def test_header_declares_expected_entry_points():
     names = _declared_symbols()
     for n in ("sqa_attn_fwd", "sqa_attn_fwd_ex", "sqa_attn_bwd", "sqa_attn_bwd_workspace_size",
               "sqa_attn_fwd_cross", "sqa_attn_bwd_cross", "sqa_attn_fwd_packed", "sqa_attn_bwd_packed",
-              "sqa_attn_fwd_window", "sqa_attn_bwd_window",
+              "sqa_attn_fwd_window", "sqa_attn_bwd_window", "sqa_attn_decode", "sqa_attn_decode_workspace_size",
               "sqa_proj", "sqa_device_status", "sqa_status_string", "sqa_version"):
         assert n in names
 
@@ -122,6 +122,30 @@ def test_window_rejects_invalid_arguments():
                                    -1, 0, 0.1, FAKE, ws, None) == sqa.SQA_ERR_INVALID_ARG
     assert lib.sqa_attn_bwd_window(FAKE, FAKE, FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1, 8, 4, 2, 32,
                                    2, 2, 0.1, FAKE, ws - 4, None) == sqa.SQA_ERR_INVALID_ARG
+
+
+def test_decode_workspace_and_invalid_arguments():
+    lib = sqa.library()
+    # One chunk per sequence (L_max <= 256): no workspace.
+    assert sqa.sqa_attn_decode_workspace_size(4, 1, 8, 4, 128, 256) == 0
+    ws = sqa.sqa_attn_decode_workspace_size(2, 1, 8, 4, 128, 32768)
+    assert ws > 0 and ws % 16 == 0
+    assert sqa.sqa_attn_decode_workspace_size(2, 4, 8, 3, 128, 100) == 0
+    assert sqa.sqa_attn_decode_workspace_size(2, 8, 8, 4, 128, 4) == 0   # L_max < n_new
+
+    def call(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, lens=FAKE, out=FAKE, od=0, lse=None, B=2, n=1, H_q=8, H_kv=4, d=128,
+                 L=32768, scale=0.1, ws=FAKE, wsb=ws)
+        a.update(kw)
+        return lib.sqa_attn_decode(a["q"], a["k"], a["v"], a["lens"], a["out"], a["od"], a["lse"], a["B"], a["n"],
+                                   a["H_q"], a["H_kv"], a["d"], a["L"], a["scale"], a["ws"], a["wsb"], None)
+
+    for kw in (dict(lens=None), dict(out=None), dict(ws=None), dict(wsb=ws - 16), dict(od=4), dict(n=0),
+               dict(L=0), dict(H_kv=3), dict(lens=FAKE + 2), dict(out=FAKE + 8)):
+        assert call(**kw) == sqa.SQA_ERR_INVALID_ARG, kw
+    assert call(d=96) == sqa.SQA_ERR_UNSUPPORTED
+    # 2 heads per group x 65 new tokens = 130 rows > one 128-row tile.
+    assert call(n=65, wsb=1 << 30) == sqa.SQA_ERR_UNSUPPORTED
 
 
 def test_packed_rejects_invalid_arguments():
