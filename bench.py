@@ -680,6 +680,22 @@ def run_profile(args):
         for _ in range(args.steps):
             sqa.sqa_attn_fwd(x["q"], x["k"], x["v"], out, B, N, H_q, H_kv, d, w["causal"], 1 / math.sqrt(d),
                              stream=stream)
+    elif args.profile == "decode":
+        c = DECODE
+        B, L, n_new, d = c["B"], c["L"], c["n_new"], c["d_head"]
+        hq, hkv = DECODE_VARIANTS["SQA"]
+        g = torch.Generator(device=dev)
+        g.manual_seed(5)
+        q = torch.randn((B, n_new, hq, d), generator=g, device=dev).to(torch.bfloat16)
+        kc = torch.randn((B, L, hkv, d), generator=g, device=dev).to(torch.bfloat16)
+        vc = torch.randn((B, L, hkv, d), generator=g, device=dev).to(torch.bfloat16)
+        lens = torch.full((B,), L, dtype=torch.int32, device=dev)
+        out = torch.empty((B, n_new, hq, d), dtype=torch.bfloat16, device=dev)
+        wsb = sqa.sqa_attn_decode_workspace_size(B, n_new, hq, hkv, d, L)
+        ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=dev)
+        for _ in range(args.steps):
+            sqa.sqa_attn_decode(q, kc, vc, lens, out, sqa.SQA_DT_BF16, None, B, n_new, hq, hkv, d, L,
+                                1 / math.sqrt(d), ws if wsb else None, wsb, stream=stream)
     else:
         flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
         time_training_step(sqa, torch, stream, flush, dev, reps=max(1, args.steps - 3))
@@ -695,9 +711,10 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["sqa", "reference"], default="sqa")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["fwd", "bwd"], default=None,
+    ap.add_argument("--profile", choices=["fwd", "bwd", "decode"], default=None,
                     help="only launch the kernels (for ncu): fwd = the bench workload's forward, "
-                         "bwd = the B=4, N=8192 causal training step; no timing, no JSON")
+                         "bwd = the B=4, N=8192 causal training step, decode = one SQA decode step of "
+                         "B=16 sequences x 32768 cached tokens; no timing, no JSON")
     args = ap.parse_args(argv)
     if args.profile:
         return run_profile(args)
