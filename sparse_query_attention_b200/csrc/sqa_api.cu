@@ -335,9 +335,11 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
       o, o_bf16, static_cast<const __nv_bfloat16*>(dout), lse, dsum, lse2, B, N, H_q, n_pad);
   if (cudaGetLastError() != cudaSuccess) return SQA_ERR_CUDA;
 
-  // 2. dK, dV (KV-outer).
+  // 2. dK, dV (KV-outer).  The statistics ride in the score MMAs unless
+  // 1 / (scale log2 e) is out of range (a zero or near-zero scale).
   {
-    auto kern = sqa::bwd_dkdv_kernel<D, GradT>;
+    const bool fold = std::fabs(p.scale_log2) >= 1e-30f;
+    auto kern = fold ? sqa::bwd_dkdv_kernel<D, GradT, true> : sqa::bwd_dkdv_kernel<D, GradT, false>;
     constexpr int smem = sqa::DkdvCfg<D>::kSmemBytes;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return SQA_ERR_CUDA;

@@ -144,9 +144,24 @@ struct DkdvCfg {
   using KV = TileGeo<D, 128>;  // resident K and V tiles
   using QT = TileGeo<D, 64>;   // streamed Q / dO sub-tiles
   static constexpr int kStages = D == 128 ? 4 : 6;
-  static constexpr int kStatBytes = 1024;                        // LSE2 (256 B) + D (256 B), 1 KB aligned
-  static constexpr int kStageBytes = 2 * QT::kBytes + kStatBytes;  // Q, dO, stats
-  static constexpr int kSmemBytes = 2 * KV::kBytes + kStages * kStageBytes + 1024;
+  // Per-query statistics folded into the score MMAs: a 16-wide K step whose
+  // A operand is 1 in columns 0-2 for every key and whose B operand holds,
+  // per query, -L2 / (scale log2 e) (resp. -D) split into three bf16 parts,
+  // so S^T and dP^T arrive from the tensor core already shifted.  Both
+  // operands use the unswizzled K-major layout: 8-row x 16-byte core
+  // matrices, K neighbours 128 B apart, 8-row groups 256 B apart.
+  static constexpr int kAugRowBytes = 32;                 // 16 bf16 per row
+  static constexpr int kAugBytes = 64 * kAugRowBytes;     // one 64-query operand
+  static constexpr int kOnesBytes = 128 * kAugRowBytes;   // the 128-key ones operand
+  static constexpr int kStatLse = 0, kStatD = 256;        // fp32 -L2, -D (TMA)
+  static constexpr int kStatAugL = 1024, kStatAugD = 1024 + kAugBytes;
+  static constexpr int kStatBytes = 1024 + 2 * kAugBytes;            // 5 KB, keeps stages 1 KB aligned
+  static constexpr int kStageBytes = 2 * QT::kBytes + kStatBytes;     // Q, dO, statistics
+  static constexpr int kSmemBytes = 2 * KV::kBytes + kStages * kStageBytes + kOnesBytes + 1024;
+  static_assert(kStageBytes % 1024 == 0, "stage alignment");
+  __host__ __device__ static constexpr uint32_t aug_off(int r, int e) {  // byte offset of element (r, e)
+    return (r / 8) * 256 + (e / 8) * 128 + (r % 8) * 16 + (e % 8) * 2;
+  }
   // Score buffers in TMEM: three when they fit next to dV and dK (d <= 64).
   static constexpr int kBufs = D <= 64 ? 3 : 2;
   // TMEM columns: S^T/P^T and dP^T/dS^T of buffer b, then dV and dK.
@@ -156,7 +171,17 @@ struct DkdvCfg {
   static_assert(kColDK + D <= 512, "TMEM columns");
 };
 
-template <int D, typename GradT>
+// Splits v into three bf16 parts whose sum is v to about 2^-24 relative.
+__device__ __forceinline__ void split3_bf16(float v, __nv_bfloat16& h, __nv_bfloat16& m, __nv_bfloat16& l) {
+  h = __float2bfloat16_rn(v);
+  const float r1 = v - __bfloat162float(h);
+  m = __float2bfloat16_rn(r1);
+  l = __float2bfloat16_rn(r1 - __bfloat162float(m));
+}
+
+// kAug: statistics folded into the score MMAs (needs a scale with a finite
+// 1 / (scale log2 e)); otherwise the softmax warps read them per column.
+template <int D, typename GradT, bool kAug>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -169,6 +194,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __shared__ __align__(8) uint64_t kv_full;
   __shared__ __align__(8) uint64_t st_full[C::kStages];
   __shared__ __align__(8) uint64_t st_empty[C::kStages];
+  __shared__ __align__(8) uint64_t aug_full[C::kStages];
   __shared__ __align__(8) uint64_t s_full[C::kBufs];
   __shared__ __align__(8) uint64_t p_ready[C::kBufs];
   __shared__ __align__(8) uint64_t mma_done;
@@ -179,6 +205,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t* k_smem = smem;
   uint8_t* v_smem = smem + KV::kBytes;
   uint8_t* stages = smem + 2 * KV::kBytes;
+  uint8_t* ones_smem = stages + C::kStages * C::kStageBytes;
 
   const int warp = warp_id_uniform();
   const int lane = threadIdx.x & 31;
@@ -199,6 +226,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&st_full[s], 1);
       mbar_init(&st_empty[s], 1);
+      mbar_init(&aug_full[s], 1);
     }
     for (int t = 0; t < C::kBufs; ++t) {
       mbar_init(&s_full[t], 1);
@@ -219,7 +247,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (warp < 4) {
   regs_dealloc<kBwdRegsLow>();
-  if (warp == 0) {
+  if (kAug && warp == 3) {
+    // ---------------- statistics operands (whole warp) ----------------
+    // The ones operand once, then per stage the three-part bf16 split of
+    // -L2 / (scale log2 e) and of -D for its 64 queries.
+    for (int i = lane; i < 128 * 2; i += 32) {
+      const int r = i >> 1, chunk = i & 1;
+      const uint4 v = chunk == 0 ? make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(ones_smem + C::aug_off(r, chunk * 8)) = v;
+    }
+    const float inv_sl2 = 1.f / p.scale_log2;
+    for (int s = 0; s < n_steps; ++s) {
+      const int st = s % C::kStages;
+      if (!mbar_wait(&st_full[st], (s / C::kStages) & 1, &abort_flag)) break;
+      uint8_t* stat = stages + st * C::kStageBytes + 2 * QT::kBytes;
+      const float* nl2 = reinterpret_cast<const float*>(stat + C::kStatLse);
+      const float* nd = reinterpret_cast<const float*>(stat + C::kStatD);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int r = lane + 32 * half;
+        __nv_bfloat16 h, m, l;
+        split3_bf16(nl2[r] * inv_sl2, h, m, l);
+        __nv_bfloat162 hm = __halves2bfloat162(h, m), l0 = __halves2bfloat162(l, __float2bfloat16_rn(0.f));
+        *reinterpret_cast<uint4*>(stat + C::kStatAugL + C::aug_off(r, 0)) =
+            make_uint4(*reinterpret_cast<uint32_t*>(&hm), *reinterpret_cast<uint32_t*>(&l0), 0u, 0u);
+        *reinterpret_cast<uint4*>(stat + C::kStatAugL + C::aug_off(r, 8)) = make_uint4(0u, 0u, 0u, 0u);
+        split3_bf16(nd[r], h, m, l);
+        hm = __halves2bfloat162(h, m);
+        l0 = __halves2bfloat162(l, __float2bfloat16_rn(0.f));
+        *reinterpret_cast<uint4*>(stat + C::kStatAugD + C::aug_off(r, 0)) =
+            make_uint4(*reinterpret_cast<uint32_t*>(&hm), *reinterpret_cast<uint32_t*>(&l0), 0u, 0u);
+        *reinterpret_cast<uint4*>(stat + C::kStatAugD + C::aug_off(r, 8)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&aug_full[st]);
+    }
+  } else if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
       mbar_arrive_expect_tx(&kv_full, 2 * KV::kBytes);
@@ -240,8 +304,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tma_load_4d(&tm_do, &st_full[st], dst + QT::kBytes + c * QT::kChunkBytes, c * QT::kRowElems, h, q0, b);
         }
         const int stat_row = b * p.H_q + h;
-        tma_load_2d(&tm_lse2, &st_full[st], dst + 2 * QT::kBytes, q0, stat_row);
-        tma_load_2d(&tm_dsum, &st_full[st], dst + 2 * QT::kBytes + 256, q0, stat_row);
+        tma_load_2d(&tm_lse2, &st_full[st], dst + 2 * QT::kBytes + C::kStatLse, q0, stat_row);
+        tma_load_2d(&tm_dsum, &st_full[st], dst + 2 * QT::kBytes + C::kStatD, q0, stat_row);
       }
       mbar_drain(&kv_full, 0);
       for (int l = max(0, s - C::kStages); l < s; ++l) mbar_drain(&st_full[l % C::kStages], (l / C::kStages) & 1);
@@ -258,6 +322,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t v_kd = KV::kmajor_base(smem_addr(v_smem));
       const uint64_t st_kd = QT::kmajor_base(smem_addr(stages));
       const uint64_t st_mn = QT::mnmajor_base(smem_addr(stages));
+      // Unswizzled K-major: leading (K) byte offset 128, stride (8-row) 256.
+      const uint64_t ones_d = smem_desc(smem_addr(ones_smem), 128, 256, kSwNone);
+      const uint64_t aug_d = smem_desc(smem_addr(stages + 2 * QT::kBytes + C::kStatAugL), 128, 256, kSwNone);
       auto issue_scores = [&](int s) {
         const int buf = s % C::kBufs;
         const uint64_t q_kd = desc_advance(st_kd, (s % C::kStages) * C::kStageBytes);
@@ -271,11 +338,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           mma_ss_w(tmem + C::col_dp(buf), desc_advance(v_kd, KV::kmajor_off(kk)),
                  desc_advance(do_kd, QT::kmajor_off(kk)), idesc_s, kk > 0);
         }
+        if constexpr (kAug) {  // + (-L2 / (scale log2 e)) and + (-D), per query column
+          const uint64_t a0 = desc_advance(aug_d, (s % C::kStages) * C::kStageBytes);
+          mma_ss_w(tmem + C::col_s(buf), ones_d, a0, idesc_s, 1u);
+          mma_ss_w(tmem + C::col_dp(buf), ones_d, desc_advance(a0, C::kAugBytes), idesc_s, 1u);
+        }
         mma_commit_w(&s_full[buf]);
+      };
+      // A stage's score MMAs need its TMA data and, folded, its statistics.
+      auto stage_ready = [&](int s) {
+        const int st = s % C::kStages;
+        const uint32_t ph = (s / C::kStages) & 1;
+        if (!mbar_wait(&st_full[st], ph, &abort_flag)) return false;
+        if constexpr (kAug) return mbar_wait(&aug_full[st], ph, &abort_flag);
+        return true;
       };
       bool ok = mbar_wait(&kv_full, 0, &abort_flag);
       for (int s = 0; s < C::kBufs && s < n_steps && ok; ++s) {
-        ok = mbar_wait(&st_full[s % C::kStages], (s / C::kStages) & 1, &abort_flag);
+        ok = stage_ready(s);
         if (ok) {
           tc_fence_after();
           issue_scores(s);
@@ -297,7 +377,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mma_commit_w(&st_empty[s % C::kStages]);
         if (s + C::kBufs < n_steps) {  // the next scores into the buffer just read
           const int s2 = s + C::kBufs;
-          if (!mbar_wait(&st_full[s2 % C::kStages], (s2 / C::kStages) & 1, &abort_flag)) break;
+          if (!stage_ready(s2)) break;
           tc_fence_after();
           issue_scores(s2);
         }
@@ -322,14 +402,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         break;
       }
       tc_fence_after();
-      uint32_t sr[64], dr[64];
-      tmem_ld32(lane_base + C::col_s(buf), *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(lane_base + C::col_s(buf) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld32(lane_base + C::col_dp(buf), *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
-      tmem_ld32(lane_base + C::col_dp(buf) + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+      const uint32_t s_col = lane_base + C::col_s(buf), dp_col = lane_base + C::col_dp(buf);
+      // Four quarters of 16 query columns, register double-buffered: the
+      // next quarter's S^T / dP^T loads are in flight while this one is
+      // computed, and each quarter's P^T / dS^T (8 packed words each) go
+      // back over columns whose scores have already been read.  Few scores
+      // are live at once, which leaves registers for the exponentials of a
+      // quarter to overlap.
+      uint32_t sa[16], da[16], sb[16], db[16];
+      tmem_ld16(s_col, sa);
+      tmem_ld16(dp_col, da);
       const uint8_t* stat = stages + (s % C::kStages) * C::kStageBytes + 2 * QT::kBytes;
-      const float* l2 = reinterpret_cast<const float*>(stat);
-      const float* dd = reinterpret_cast<const float*>(stat + 256);
+      const float* l2 = reinterpret_cast<const float*>(stat + C::kStatLse);
+      const float* dd = reinterpret_cast<const float*>(stat + C::kStatD);
       const int q0 = (qs_begin + s % per_head) * 64;
       // Query column c (token q0 + c) contributes iff q0 + c < N and key u
       // is inside its band: u - win_r <= q0 + c <= u + win_l.  Full tiles
@@ -340,28 +425,54 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         hi = min(hi, u + p.win_l - q0 + 1);
       }
       const bool full = __all_sync(0xffffffffu, lo <= 0 && hi >= 64);
-      tmem_wait_ld();
-      uint32_t pk[32], dk[32];
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
+      tmem_wait_ld();
+      reg_fence16(sa);
+      reg_fence16(da);
       // P = 2^(s sl2 - L2), dS = P (dP - D), two columns per packed op; the
       // workspace holds -L2 and -D.  A quarter of the exponentials run as
       // the FMA-pipe polynomial.
-      auto body = [&](auto masked) {
+      // Folded statistics (kAug): the scores arrive as S^T - L2 / (scale
+      // log2 e) and dP^T - D.  Otherwise the quarter's -L2 and -D come as
+      // 16-byte shared-memory loads issued one quarter ahead (shared-memory
+      // loads of these broadcast values are what kept this loop waiting,
+      // hence the folding).
+      auto stats = [&](int qt, float4(&lq)[4], float4(&dq4)[4]) {
+        if constexpr (!kAug) {
 #pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) {
-          const int c = 2 * c2;
-          const float2 nl = *reinterpret_cast<const float2*>(l2 + c);
-          const float2 nd = *reinterpret_cast<const float2*>(dd + c);
+          for (int k = 0; k < 4; ++k) {
+            lq[k] = *reinterpret_cast<const float4*>(l2 + qt * 16 + 4 * k);
+            dq4[k] = *reinterpret_cast<const float4*>(dd + qt * 16 + 4 * k);
+          }
+        }
+      };
+      auto quarter = [&](auto qtc, const uint32_t(&sr)[16], const uint32_t(&dr)[16], const float4(&lq)[4],
+                         const float4(&dq4)[4], auto masked) {
+        constexpr int qt = decltype(qtc)::value;
+        uint32_t pk[8], dk[8];
+#pragma unroll
+        for (int c2 = 0; c2 < 8; ++c2) {
+          const int c = qt * 16 + 2 * c2;  // query column of the pair
           float x0, x1, p0, p1, d0, d1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, f2_pack(nl.x, nl.y)),
-                    x0, x1);
+          const uint64_t sp = f2_pack(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1]));
+          const uint64_t dp = f2_pack(__uint_as_float(dr[2 * c2]), __uint_as_float(dr[2 * c2 + 1]));
+          uint64_t t;  // dP - D
+          if constexpr (kAug) {
+            f2_unpack(f2_mul(sp, sl2x2), x0, x1);
+            t = dp;
+          } else {
+            const float4 l4 = lq[c2 >> 1], d4 = dq4[c2 >> 1];
+            const float2 nl = (c2 & 1) ? make_float2(l4.z, l4.w) : make_float2(l4.x, l4.y);
+            const float2 nd = (c2 & 1) ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
+            f2_unpack(f2_fma(sp, sl2x2, f2_pack(nl.x, nl.y)), x0, x1);
+            t = f2_add(dp, f2_pack(nd.x, nd.y));
+          }
           if ((c2 & 3) == 3) {
             exp2_poly_pair(x0, x1, p0, p1);
           } else {
             p0 = ex2_approx(x0);
             p1 = ex2_approx(x1);
           }
-          const uint64_t t = f2_add(f2_pack(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])), f2_pack(nd.x, nd.y));
           f2_unpack(f2_mul(f2_pack(p0, p1), t), d0, d1);
           if constexpr (decltype(masked)::value) {
             const bool k0 = c >= lo && c < hi, k1 = c + 1 >= lo && c + 1 < hi;
@@ -373,13 +484,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           pk[c2] = pack_bf16x2(p0, p1);
           dk[c2] = pack_bf16x2(d0, d1);
         }
+        tmem_st8(s_col + qt * 8, pk);
+        tmem_st8(dp_col + qt * 8, dk);
+      };
+      auto all_quarters = [&](auto masked) {
+        float4 la[4], dla[4], lb[4], dlb[4];
+        stats(0, la, dla);
+        tmem_ld16(s_col + 16, sb);
+        tmem_ld16(dp_col + 16, db);
+        stats(1, lb, dlb);
+        quarter(IntC<0>{}, sa, da, la, dla, masked);
+        tmem_wait_ld();
+        reg_fence16(sb);
+        reg_fence16(db);
+        tmem_ld16(s_col + 32, sa);
+        tmem_ld16(dp_col + 32, da);
+        stats(2, la, dla);
+        quarter(IntC<1>{}, sb, db, lb, dlb, masked);
+        tmem_wait_ld();
+        reg_fence16(sa);
+        reg_fence16(da);
+        tmem_ld16(s_col + 48, sb);
+        tmem_ld16(dp_col + 48, db);
+        stats(3, lb, dlb);
+        quarter(IntC<2>{}, sa, da, la, dla, masked);
+        tmem_wait_ld();
+        reg_fence16(sb);
+        reg_fence16(db);
+        quarter(IntC<3>{}, sb, db, lb, dlb, masked);
       };
       if (full)
-        body(BoolC<false>{});
+        all_quarters(BoolC<false>{});
       else
-        body(BoolC<true>{});
-      tmem_st32(lane_base + C::col_s(buf), pk);
-      tmem_st32(lane_base + C::col_dp(buf), dk);
+        all_quarters(BoolC<true>{});
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -596,11 +733,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         break;
       }
       tc_fence_after();
-      uint32_t sr[64], dr[64];
-      tmem_ld32(lane_base + C::col_s(buf), *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(lane_base + C::col_s(buf) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld32(lane_base + C::col_dp(buf), *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
-      tmem_ld32(lane_base + C::col_dp(buf) + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+      const uint32_t s_col = lane_base + C::col_s(buf), dp_col = lane_base + C::col_dp(buf);
+      // Four register double-buffered quarters of 16 keys, as in the dK/dV
+      // kernel: loads of the next quarter overlap this one's arithmetic and
+      // each quarter's dS (8 packed words) goes back over scores already read.
+      uint32_t sa[16], da[16], sb[16], db[16];
+      tmem_ld16(s_col, sa);
+      tmem_ld16(dp_col, da);
       const int kbase = (ks_begin + s) * 64;
       int lo = 0, hi = p.Nkv - kbase;  // keys [lo, hi) of the sub-tile are visible
       if (p.masked) {
@@ -609,23 +748,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       const bool full = __all_sync(0xffffffffu, lo <= 0 && hi >= 64);
       tmem_wait_ld();
-      uint32_t dk[32];
+      reg_fence16(sa);
+      reg_fence16(da);
       // dS = 2^(s sl2 - L2) (dP - D) with the row's -L2 and -D (nl2, ndd),
       // two keys per packed op, a quarter of the exponentials as the
       // FMA-pipe polynomial; full tiles skip the per-element key test.
-      auto body = [&](auto masked) {
+      auto quarter = [&](auto qtc, const uint32_t(&sr)[16], const uint32_t(&dr)[16], auto masked) {
+        constexpr int qt = decltype(qtc)::value;
+        uint32_t dk[8];
 #pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) {
-          const int c = 2 * c2;
+        for (int c2 = 0; c2 < 8; ++c2) {
+          const int c = qt * 16 + 2 * c2;  // key column of the pair
           float x0, x1, p0, p1, d0, d1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, nl2x2), x0, x1);
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1])), sl2x2, nl2x2), x0,
+                    x1);
           if ((c2 & 3) == 3) {
             exp2_poly_pair(x0, x1, p0, p1);
           } else {
             p0 = ex2_approx(x0);
             p1 = ex2_approx(x1);
           }
-          const uint64_t t = f2_add(f2_pack(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])), ndd2);
+          const uint64_t t = f2_add(f2_pack(__uint_as_float(dr[2 * c2]), __uint_as_float(dr[2 * c2 + 1])), ndd2);
           f2_unpack(f2_mul(f2_pack(p0, p1), t), d0, d1);
           if constexpr (decltype(masked)::value) {
             d0 = (c >= lo && c < hi) ? d0 : 0.f;
@@ -633,12 +776,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           dk[c2] = pack_bf16x2(d0, d1);
         }
+        tmem_st8(s_col + qt * 8, dk);
+      };
+      auto all_quarters = [&](auto masked) {
+        tmem_ld16(s_col + 16, sb);
+        tmem_ld16(dp_col + 16, db);
+        quarter(IntC<0>{}, sa, da, masked);
+        tmem_wait_ld();
+        reg_fence16(sb);
+        reg_fence16(db);
+        tmem_ld16(s_col + 32, sa);
+        tmem_ld16(dp_col + 32, da);
+        quarter(IntC<1>{}, sb, db, masked);
+        tmem_wait_ld();
+        reg_fence16(sa);
+        reg_fence16(da);
+        tmem_ld16(s_col + 48, sb);
+        tmem_ld16(dp_col + 48, db);
+        quarter(IntC<2>{}, sa, da, masked);
+        tmem_wait_ld();
+        reg_fence16(sb);
+        reg_fence16(db);
+        quarter(IntC<3>{}, sb, db, masked);
       };
       if (full)
-        body(BoolC<false>{});
+        all_quarters(BoolC<false>{});
       else
-        body(BoolC<true>{});
-      tmem_st32(lane_base + C::col_s(buf), dk);
+        all_quarters(BoolC<true>{});
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();

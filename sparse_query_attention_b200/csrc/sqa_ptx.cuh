@@ -403,6 +403,20 @@ template <bool B>
 struct BoolC {
   static constexpr bool value = B;
 };
+template <int V>
+struct IntC {
+  static constexpr int value = V;
+};
+
+// Ties registers written by an earlier tcgen05.ld to a point after
+// tcgen05.wait::ld: the empty volatile asm "redefines" them, so no consumer
+// can be scheduled above the wait (both asm statements keep their order).
+__device__ __forceinline__ void reg_fence16(uint32_t (&r)[16]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]));
+}
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
