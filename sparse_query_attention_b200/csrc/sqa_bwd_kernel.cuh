@@ -346,12 +346,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mma_commit_w(&s_full[buf]);
       };
       // A stage's score MMAs need its TMA data and, folded, its statistics.
+      // With folded statistics one wait suffices: the statistics warp
+      // arrives on aug_full only after it has seen st_full, and that arrive
+      // releases what the TMA wrote along with its own stores.
       auto stage_ready = [&](int s) {
         const int st = s % C::kStages;
         const uint32_t ph = (s / C::kStages) & 1;
-        if (!mbar_wait(&st_full[st], ph, &abort_flag)) return false;
         if constexpr (kAug) return mbar_wait(&aug_full[st], ph, &abort_flag);
-        return true;
+        return mbar_wait(&st_full[st], ph, &abort_flag);
       };
       bool ok = mbar_wait(&kv_full, 0, &abort_flag);
       for (int s = 0; s < C::kBufs && s < n_steps && ok; ++s) {
