@@ -148,6 +148,26 @@ def test_decode_workspace_and_invalid_arguments():
     assert call(n=65, wsb=1 << 30) == sqa.SQA_ERR_UNSUPPORTED
 
 
+def test_size_limits_are_rejected_before_launch():
+    """Shapes past the kernels' 32-bit index ranges return
+    SQA_ERR_UNSUPPORTED from the host checks (nothing is launched, so fake
+    pointers are safe here)."""
+    lib = sqa.library()
+    # B * N * H_q rows at 2^31.
+    assert _fwd(B=1, N=1 << 28, H_q=8, H_kv=4, causal=0) == sqa.SQA_ERR_UNSUPPORTED
+    assert _fwd(B=2, N=1 << 27, H_q=8, H_kv=8, causal=0) == sqa.SQA_ERR_UNSUPPORTED
+    # A band (causal or window) needs N <= 2^30.
+    assert lib.sqa_attn_fwd_window(FAKE, FAKE, FAKE, FAKE, 0, None, 1, (1 << 30) + 64, 1, 1, 32, 5, 0, 0.1,
+                                   None) == sqa.SQA_ERR_UNSUPPORTED
+    # Key rows B * N_kv * H_kv at 2^31 for cross attention.
+    assert lib.sqa_attn_fwd_cross(FAKE, FAKE, FAKE, FAKE, 0, None, 1, 16, 1 << 29, 4, 4, 32, 0.1,
+                                  None) == sqa.SQA_ERR_UNSUPPORTED
+    # Decode caches of B * L_max * H_kv >= 2^31 rows.
+    ws = sqa.sqa_attn_decode_workspace_size(2, 1, 8, 8, 64, 1 << 27)
+    assert lib.sqa_attn_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 0, None, 2, 1, 8, 8, 64, 1 << 27, 0.1, FAKE, ws,
+                               None) == sqa.SQA_ERR_UNSUPPORTED
+
+
 def test_packed_rejects_invalid_arguments():
     lib = sqa.library()
     assert lib.sqa_attn_fwd_packed(None, FAKE, 0, None, 1, 8, 4, 2, 32, 1, 0.1, None) == sqa.SQA_ERR_INVALID_ARG
