@@ -128,32 +128,57 @@ def sqa_status_string(status: int) -> str:
     return status_string(status)
 
 
+_BF, _F32, _I32, _U8 = "torch.bfloat16", "torch.float32", "torch.int32", "torch.uint8"
+_DT = {SQA_DT_F32: _F32, SQA_DT_BF16: _BF}
+
+
+def _t(x, dtype, numel, name):
+    """_ptr with the checks the C ABI cannot make: a torch tensor must have
+    the element type the call reads or writes and at least the elements the
+    shape arguments imply (integers and None pass through unchecked)."""
+    if x is not None and not isinstance(x, int):
+        if dtype is not None and str(x.dtype) != dtype:
+            raise ValueError(f"{name}: expected {dtype}, got {x.dtype}")
+        if numel > 0 and x.numel() < numel:
+            raise ValueError(f"{name}: {x.numel()} elements, the shape needs {numel}")
+    return _ptr(x)
+
+
 def sqa_attn_fwd(q, k, v, out, B, N, H_q, H_kv, d_head, causal, scale, stream=None) -> None:
-    _check(library().sqa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, N, H_q, H_kv, d_head,
-                             int(bool(causal)), float(scale), _stream(stream)), "sqa_attn_fwd")
+    nq, nkv = B * N * H_q * d_head, B * N * H_kv * d_head
+    _check(library().sqa_attn_fwd(_t(q, _BF, nq, "q"), _t(k, _BF, nkv, "k"), _t(v, _BF, nkv, "v"),
+                                  _t(out, _F32, nq, "out"), B, N, H_q, H_kv, d_head, int(bool(causal)),
+                                  float(scale), _stream(stream)), "sqa_attn_fwd")
 
 
 def sqa_attn_fwd_ex(q, k, v, out, out_dtype, lse, B, N, H_q, H_kv, d_head, causal, scale,
                     stream=None) -> None:
-    _check(library().sqa_attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(out_dtype), _ptr(lse),
-                                B, N, H_q, H_kv, d_head, int(bool(causal)), float(scale),
-                                _stream(stream)), "sqa_attn_fwd_ex")
+    nq, nkv = B * N * H_q * d_head, B * N * H_kv * d_head
+    _check(library().sqa_attn_fwd_ex(_t(q, _BF, nq, "q"), _t(k, _BF, nkv, "k"), _t(v, _BF, nkv, "v"),
+                                     _t(out, _DT.get(out_dtype), nq, "out"), int(out_dtype),
+                                     _t(lse, _F32, B * H_q * N, "lse"), B, N, H_q, H_kv, d_head, int(bool(causal)),
+                                     float(scale), _stream(stream)), "sqa_attn_fwd_ex")
 
 
 def sqa_attn_fwd_cross(q, k, v, out, out_dtype, lse, B, N_q, N_kv, H_q, H_kv, d_head, scale,
                        stream=None) -> None:
     """Cross / memory attention: N_q queries, N_kv keys, no mask."""
-    _check(library().sqa_attn_fwd_cross(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(out_dtype), _ptr(lse),
-                                        B, N_q, N_kv, H_q, H_kv, d_head, float(scale),
-                                        _stream(stream)), "sqa_attn_fwd_cross")
+    nq, nkv = B * N_q * H_q * d_head, B * N_kv * H_kv * d_head
+    _check(library().sqa_attn_fwd_cross(_t(q, _BF, nq, "q"), _t(k, _BF, nkv, "k"), _t(v, _BF, nkv, "v"),
+                                        _t(out, _DT.get(out_dtype), nq, "out"), int(out_dtype),
+                                        _t(lse, _F32, B * H_q * N_q, "lse"), B, N_q, N_kv, H_q, H_kv, d_head,
+                                        float(scale), _stream(stream)), "sqa_attn_fwd_cross")
 
 
 def sqa_attn_fwd_window(q, k, v, out, out_dtype, lse, B, N, H_q, H_kv, d_head, window_left, window_right,
                         scale, stream=None) -> None:
     """Sliding-window forward: query t sees keys t - left .. t + right."""
-    _check(library().sqa_attn_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(out_dtype), _ptr(lse),
-                                         B, N, H_q, H_kv, d_head, int(window_left), int(window_right),
-                                         float(scale), _stream(stream)), "sqa_attn_fwd_window")
+    nq, nkv = B * N * H_q * d_head, B * N * H_kv * d_head
+    _check(library().sqa_attn_fwd_window(_t(q, _BF, nq, "q"), _t(k, _BF, nkv, "k"), _t(v, _BF, nkv, "v"),
+                                         _t(out, _DT.get(out_dtype), nq, "out"), int(out_dtype),
+                                         _t(lse, _F32, B * H_q * N, "lse"), B, N, H_q, H_kv, d_head,
+                                         int(window_left), int(window_right), float(scale), _stream(stream)),
+           "sqa_attn_fwd_window")
 
 
 def sqa_attn_decode_workspace_size(B, n_new, H_q, H_kv, d_head, L_max) -> int:
@@ -164,59 +189,75 @@ def sqa_attn_decode(q, k_cache, v_cache, cache_lens, out, out_dtype, lse, B, n_n
                     scale, workspace, workspace_bytes, stream=None) -> None:
     """Decode n_new tokens per sequence against a KV cache; cache_lens is a
     device int32 tensor [B]."""
-    _check(library().sqa_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_lens), _ptr(out),
-                                     int(out_dtype), _ptr(lse), B, n_new, H_q, H_kv, d_head, L_max, float(scale),
-                                     _ptr(workspace), int(workspace_bytes), _stream(stream)), "sqa_attn_decode")
+    nq, nc = B * n_new * H_q * d_head, B * L_max * H_kv * d_head
+    _check(library().sqa_attn_decode(_t(q, _BF, nq, "q"), _t(k_cache, _BF, nc, "k_cache"),
+                                     _t(v_cache, _BF, nc, "v_cache"), _t(cache_lens, _I32, B, "cache_lens"),
+                                     _t(out, _DT.get(out_dtype), nq, "out"), int(out_dtype),
+                                     _t(lse, _F32, B * H_q * n_new, "lse"), B, n_new, H_q, H_kv, d_head, L_max,
+                                     float(scale), _t(workspace, _U8, int(workspace_bytes), "workspace"),
+                                     int(workspace_bytes), _stream(stream)), "sqa_attn_decode")
 
 
 def sqa_attn_fwd_packed(qkv, out, out_dtype, lse, B, N, H_q, H_kv, d_head, causal, scale,
                         stream=None) -> None:
     """Forward on a packed QKV buffer [B, N, H_q + 2*H_kv, d_head]."""
-    _check(library().sqa_attn_fwd_packed(_ptr(qkv), _ptr(out), int(out_dtype), _ptr(lse), B, N, H_q, H_kv,
-                                         d_head, int(bool(causal)), float(scale), _stream(stream)),
-           "sqa_attn_fwd_packed")
+    _check(library().sqa_attn_fwd_packed(_t(qkv, _BF, B * N * (H_q + 2 * H_kv) * d_head, "qkv"),
+                                         _t(out, _DT.get(out_dtype), B * N * H_q * d_head, "out"), int(out_dtype),
+                                         _t(lse, _F32, B * H_q * N, "lse"), B, N, H_q, H_kv, d_head,
+                                         int(bool(causal)), float(scale), _stream(stream)), "sqa_attn_fwd_packed")
 
 
 def sqa_attn_bwd_workspace_size(B, N, H_q, H_kv, d_head) -> int:
     return int(library().sqa_attn_bwd_workspace_size(B, N, H_q, H_kv, d_head))
 
 
+def _bwd_args(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B, N_q, N_kv, H_q, H_kv, d_head):
+    nq, nkv = B * N_q * H_q * d_head, B * N_kv * H_kv * d_head
+    g = _DT.get(grad_dtype)
+    return (_t(q, _BF, nq, "q"), _t(k, _BF, nkv, "k"), _t(v, _BF, nkv, "v"), _t(out, _DT.get(o_dtype), nq, "out"),
+            int(o_dtype), _t(dout, _BF, nq, "dout"), _t(lse, _F32, B * H_q * N_q, "lse"), _t(dq, g, nq, "dq"),
+            _t(dk, g, nkv, "dk"), _t(dv, g, nkv, "dv"), int(grad_dtype))
+
+
 def sqa_attn_bwd(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B, N, H_q, H_kv,
                  d_head, causal, scale, workspace, workspace_bytes, stream=None) -> None:
-    _check(library().sqa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(o_dtype), _ptr(dout),
-                             _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), int(grad_dtype),
-                             B, N, H_q, H_kv, d_head, int(bool(causal)), float(scale),
-                             _ptr(workspace), int(workspace_bytes), _stream(stream)),
-           "sqa_attn_bwd")
+    _check(library().sqa_attn_bwd(*_bwd_args(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B, N, N,
+                                             H_q, H_kv, d_head),
+                                  B, N, H_q, H_kv, d_head, int(bool(causal)), float(scale),
+                                  _t(workspace, _U8, int(workspace_bytes), "workspace"), int(workspace_bytes),
+                                  _stream(stream)), "sqa_attn_bwd")
 
 
 def sqa_attn_bwd_cross(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B, N_q, N_kv, H_q,
                        H_kv, d_head, scale, workspace, workspace_bytes, stream=None) -> None:
     """Gradient of sqa_attn_fwd_cross; workspace sized for N_q query rows."""
-    _check(library().sqa_attn_bwd_cross(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(o_dtype), _ptr(dout),
-                                        _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), int(grad_dtype),
+    _check(library().sqa_attn_bwd_cross(*_bwd_args(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B,
+                                                   N_q, N_kv, H_q, H_kv, d_head),
                                         B, N_q, N_kv, H_q, H_kv, d_head, float(scale),
-                                        _ptr(workspace), int(workspace_bytes), _stream(stream)),
-           "sqa_attn_bwd_cross")
+                                        _t(workspace, _U8, int(workspace_bytes), "workspace"), int(workspace_bytes),
+                                        _stream(stream)), "sqa_attn_bwd_cross")
 
 
 def sqa_attn_bwd_window(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B, N, H_q, H_kv, d_head,
                         window_left, window_right, scale, workspace, workspace_bytes, stream=None) -> None:
     """Gradient of sqa_attn_fwd_window (same window)."""
-    _check(library().sqa_attn_bwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(o_dtype), _ptr(dout),
-                                         _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), int(grad_dtype),
+    _check(library().sqa_attn_bwd_window(*_bwd_args(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B,
+                                                    N, N, H_q, H_kv, d_head),
                                          B, N, H_q, H_kv, d_head, int(window_left), int(window_right),
-                                         float(scale), _ptr(workspace), int(workspace_bytes), _stream(stream)),
-           "sqa_attn_bwd_window")
+                                         float(scale), _t(workspace, _U8, int(workspace_bytes), "workspace"),
+                                         int(workspace_bytes), _stream(stream)), "sqa_attn_bwd_window")
 
 
 def sqa_attn_bwd_packed(qkv, out, o_dtype, dout, lse, dqkv, grad_dtype, B, N, H_q, H_kv, d_head, causal,
                         scale, workspace, workspace_bytes, stream=None) -> None:
     """Gradient of sqa_attn_fwd_packed into a packed dQKV buffer."""
-    _check(library().sqa_attn_bwd_packed(_ptr(qkv), _ptr(out), int(o_dtype), _ptr(dout), _ptr(lse), _ptr(dqkv),
-                                         int(grad_dtype), B, N, H_q, H_kv, d_head, int(bool(causal)),
-                                         float(scale), _ptr(workspace), int(workspace_bytes), _stream(stream)),
-           "sqa_attn_bwd_packed")
+    nq, npk = B * N * H_q * d_head, B * N * (H_q + 2 * H_kv) * d_head
+    _check(library().sqa_attn_bwd_packed(_t(qkv, _BF, npk, "qkv"), _t(out, _DT.get(o_dtype), nq, "out"),
+                                         int(o_dtype), _t(dout, _BF, nq, "dout"), _t(lse, _F32, B * H_q * N, "lse"),
+                                         _t(dqkv, _DT.get(grad_dtype), npk, "dqkv"), int(grad_dtype),
+                                         B, N, H_q, H_kv, d_head, int(bool(causal)), float(scale),
+                                         _t(workspace, _U8, int(workspace_bytes), "workspace"), int(workspace_bytes),
+                                         _stream(stream)), "sqa_attn_bwd_packed")
 
 
 def sqa_attn_bwd_static(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B, N, H_q, H_kv,
@@ -224,19 +265,21 @@ def sqa_attn_bwd_static(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype
     """sqa_attn_bwd with the library's fixed device scratch instead of a
     caller workspace, for callers that cannot allocate device memory; see
     include/sqa.h for its size limit and sharing rules."""
-    _check(library().sqa_attn_bwd_static(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(o_dtype), _ptr(dout),
-                                    _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), int(grad_dtype),
-                                    B, N, H_q, H_kv, d_head, int(bool(causal)), float(scale),
-                                    _stream(stream)), "sqa_attn_bwd_static")
+    _check(library().sqa_attn_bwd_static(*_bwd_args(q, k, v, out, o_dtype, dout, lse, dq, dk, dv, grad_dtype, B,
+                                                    N, N, H_q, H_kv, d_head),
+                                         B, N, H_q, H_kv, d_head, int(bool(causal)), float(scale),
+                                         _stream(stream)), "sqa_attn_bwd_static")
 
 
 def sqa_proj(x, w, bias, y, y_dtype, M, K, Nout, stream=None) -> None:
-    _check(library().sqa_proj(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), int(y_dtype), M, K, Nout,
-                         _stream(stream)), "sqa_proj")
+    _check(library().sqa_proj(_t(x, _BF, M * K, "x"), _t(w, _BF, Nout * K, "w"), _t(bias, _F32, Nout, "bias"),
+                              _t(y, _DT.get(y_dtype), M * Nout, "y"), int(y_dtype), M, K, Nout, _stream(stream)),
+           "sqa_proj")
 
 
 def sqa_gemm(a, a_layout, b, b_layout, bias, c, c_dtype, accumulate, M, N, K, stream=None) -> None:
-    _check(library().sqa_gemm(_ptr(a), int(a_layout), _ptr(b), int(b_layout), _ptr(bias), _ptr(c), int(c_dtype),
+    _check(library().sqa_gemm(_t(a, _BF, M * K, "a"), int(a_layout), _t(b, _BF, N * K, "b"), int(b_layout),
+                              _t(bias, _F32, N, "bias"), _t(c, _DT.get(c_dtype), M * N, "c"), int(c_dtype),
                               int(bool(accumulate)), M, N, K, _stream(stream)), "sqa_gemm")
 
 

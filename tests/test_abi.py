@@ -201,3 +201,19 @@ def test_binding_raises_on_error_status():
     with pytest.raises(sqa.SQAError) as e:
         sqa.sqa_attn_fwd(FAKE, FAKE, FAKE, FAKE, 1, 8, 4, 3, 32, True, 0.1, stream=0)
     assert e.value.status == sqa.SQA_ERR_INVALID_ARG
+
+
+def test_binding_checks_tensor_dtype_and_size():
+    """The binding rejects tensors of the wrong element type or too few
+    elements before calling the library (CPU tensors reach these checks
+    first; a CUDA tensor is needed only to get past them)."""
+    import torch
+    q = torch.zeros(2 * 8 * 4 * 32, dtype=torch.float32)
+    with pytest.raises(ValueError, match="expected torch.bfloat16"):
+        sqa.sqa_attn_fwd(q, FAKE, FAKE, FAKE, 2, 8, 4, 2, 32, True, 0.1, stream=0)
+    small = torch.zeros(10, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="elements"):
+        sqa.sqa_attn_fwd(small, FAKE, FAKE, FAKE, 2, 8, 4, 2, 32, True, 0.1, stream=0)
+    lens = torch.zeros(3, dtype=torch.int64)
+    with pytest.raises(ValueError, match="expected torch.int32"):
+        sqa.sqa_attn_decode(FAKE, FAKE, FAKE, lens, FAKE, 0, None, 3, 1, 4, 2, 32, 64, 0.1, None, 0, stream=0)
