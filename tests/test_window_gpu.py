@@ -99,3 +99,45 @@ def test_window_n_zero_is_the_causal_path(sqa):
     torch.cuda.synchronize()
     assert torch.equal(o, o2) and torch.equal(lse, lse2)
     assert torch.equal(dq, dq2) and torch.equal(dk, dk2) and torch.equal(dv, dv2)
+
+
+@pytest.mark.parametrize("left,right", [(4095, 0), (2048, 2048)])
+def test_window_full_size_sampled_rows(sqa, left, right):
+    """The bench's sliding-window workload (B=1, N=131072, SQA (8,4), d=128):
+    128 sampled query rows of every head against the oracle."""
+    from sqa_inputs import sample_rows
+    B, N, H_q, H_kv, d = 1, 131072, 8, 4, 128
+    x = attention_inputs(B, N, H_q, H_kv, d, seed=3, device="cuda")
+    o, lse = _fwd(sqa, x, left, right)
+    torch.cuda.synchronize()
+    sqa.sqa_device_status()
+    rows = sample_rows(N, 128, seed=left + right)
+    ro, rl = attention_forward(f64(x["q"]), f64(x["k"]), f64(x["v"]), False, 1 / math.sqrt(d), rows=rows,
+                               window=(left, right))
+    assert_close(f64(o[:, rows]), ro, "O rows")
+    assert_close(f64(lse[:, :, rows]), rl, "LSE rows")
+
+
+def test_window_backward_full_size_identities(sqa):
+    """The SQA training step of the bench's causal window (N=131072, window
+    4096, d=128), checked by identities that hold at any size: every softmax
+    row sums to one, so sum_u dV[u, j] = sum over tokens and the group's
+    heads of dO, and sum_u dS[t, u] = 0, so sum_u dK[u, j] = 0.  The kernel
+    rounds P and dS to bf16 (2^-9 ~ 2e-3 relative per element).  P's rounding
+    barely moves the dV identity (measured 5e-5 relative); dS rounding leaves
+    sum_u dK at about one bf16 unit of the root-sum-square of the dK rows
+    (measured 2.4e-3).  Bounds: 1e-3 and 1e-2."""
+    B, N, H_q, H_kv, d, left = 1, 131072, 8, 4, 128, 4095
+    x = attention_inputs(B, N, H_q, H_kv, d, seed=3, with_dout=True, device="cuda")
+    o, lse = _fwd(sqa, x, left, 0)
+    dq, dk, dv = _bwd(sqa, x, o, lse, left, 0)
+    torch.cuda.synchronize()
+    sqa.sqa_device_status()
+    G = H_q // H_kv
+    do_group = x["do"].double().reshape(B, N, H_kv, G, d).sum(dim=(1, 3))  # [B, H_kv, d]
+    sv = dv.double().sum(dim=1)
+    rel_v = float((sv - do_group).norm() / do_group.norm())
+    sk = dk.double().sum(dim=1)
+    rel_k = float(sk.norm() / dk.double().norm(dim=-1).pow(2).sum().sqrt())
+    assert rel_v <= 1e-3, rel_v
+    assert rel_k <= 1e-2, rel_k
