@@ -63,6 +63,15 @@ sqa_status_t launch_status() {
 
 bool supported_d(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 
+// Streaming multiprocessors of the current device (looked up per call; the
+// attribute query is cheap and the current device may change).
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
 sqa_status_t check_attn_args(const void* q, const void* k, const void* v, int B, int N, int H_q, int H_kv, int d,
                              float scale) {
   if (!q || !k || !v) return SQA_ERR_INVALID_ARG;
@@ -401,8 +410,12 @@ sqa_status_t launch_gemm_bn(const CUtensorMap& ma, const CUtensorMap& mb, const 
   constexpr int smem = sqa::ProjSmem<BN>::kDynamicBytes;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return SQA_ERR_CUDA;
-  dim3 grid((M + kProjBM - 1) / kProjBM, (N + BN - 1) / BN);
-  kern<<<grid, 128, smem, st>>>(ma, mb, bias, c, M, K, N, accumulate);
+  // Persistent: one CTA per SM (or per tile when there are fewer tiles).
+  const long long tiles = static_cast<long long>((M + kProjBM - 1) / kProjBM) * ((N + BN - 1) / BN);
+  const int sms = num_sms();
+  if (sms <= 0) return SQA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
+  kern<<<grid, sqa::kProjThreads, smem, st>>>(ma, mb, bias, c, M, K, N, accumulate);
   return launch_status();
 }
 

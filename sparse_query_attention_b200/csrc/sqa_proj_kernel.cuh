@@ -10,13 +10,21 @@
 // MN-contiguous (A[k][m], B[k][n]), and read with the matching shared-memory
 // operand layout, so no transpose ever goes through memory.
 //
-// Design: one CTA per 128 x BN output tile, four warps.
+// Design: a persistent kernel, one CTA per SM walking the 128 x BN output
+// tiles in groups of kProjGroupM row tiles (N fastest inside a group, so the
+// CTAs running together reuse a few A row tiles and the B tiles from L2
+// instead of streaming A once per column tile), eight warps:
 //   warp 0 / one lane : TMA producer, 64-wide K slices of A and B into a
-//                       4-stage ring (128-byte swizzle).
-//   warp 1            : issues tcgen05.mma (M=128, N=BN, K=16) into a TMEM
-//                       accumulator from warp-uniform code (lane 0 issues),
-//                       commits each stage back to the producer.
-//   all four warps    : epilogue, TMEM -> registers (+C, +bias) -> global.
+//                       4-stage ring (128-byte swizzle) that runs on across
+//                       tiles.
+//   warp 1            : issues tcgen05.mma (M=128, N=BN, K=16) from
+//                       warp-uniform code (lane 0 issues) into one of two
+//                       TMEM accumulators, alternating per tile, and commits
+//                       each stage back to the producer.
+//   warp 2            : TMEM allocation.
+//   warps 4-7         : epilogue of the previous tile, TMEM -> registers
+//                       (+C, +bias) -> global, while the next tile's
+//                       mainloop runs into the other accumulator.
 #pragma once
 
 #include "sqa_ptx.cuh"
@@ -38,18 +46,36 @@ struct ProjSmem {
 // kAMN / kBMN: operand stored MN-contiguous (A[k][m] / B[k][n]) instead of
 // K-contiguous (A[m][k] / B[n][k]).  An MN-contiguous tile is loaded as
 // 64 (MN) x 64 (K) boxes, one 8 KB chunk per 64 rows of M or N.
+constexpr int kProjThreads = 256;
+constexpr int kProjGroupM = 8;  // row tiles per raster group
+
+// Output tile of linear index `tile`: groups of kProjGroupM row tiles, all
+// column tiles of a group before the next group, rows fastest inside it.
+__device__ __forceinline__ void proj_tile_coords(int tile, int m_tiles, int n_tiles, int& mt, int& nt) {
+  const int per_group = kProjGroupM * n_tiles;
+  const int group = tile / per_group;
+  const int first = group * kProjGroupM;
+  const int gm = min(kProjGroupM, m_tiles - first);
+  const int local = tile - group * per_group;
+  mt = first + local % gm;
+  nt = local / gm;
+}
+
 template <int BN, bool kOutBf16, bool kAMN, bool kBMN>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kProjThreads, 1)
     proj_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                      const float* __restrict__ bias, void* __restrict__ y, int M, int K, int Nout, int accumulate) {
   static_assert(!kBMN || BN % 64 == 0, "MN-contiguous B needs BN in 64, 128, 256");
   using S = ProjSmem<BN>;
-  constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
-  constexpr uint32_t kMnChunk = 64 * 128;  // one 64 x 64 MN-contiguous box
+  constexpr uint32_t kAccCols = BN < 32 ? 32 : BN;  // one accumulator
+  constexpr uint32_t kTmemCols = 2 * kAccCols;        // two, alternating per tile
+  constexpr uint32_t kMnChunk = 64 * 128;             // one 64 x 64 MN-contiguous box
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kProjStages];
   __shared__ __align__(8) uint64_t empty_bar[kProjStages];
-  __shared__ __align__(8) uint64_t acc_bar;
+  __shared__ __align__(8) uint64_t acc_full[2];
+  __shared__ __align__(8) uint64_t acc_empty[2];
+  __shared__ __align__(8) uint64_t mma_done;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
 
@@ -59,8 +85,9 @@ __global__ void __launch_bounds__(128, 1)
 
   const int warp = warp_id_uniform();
   const int lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kProjBM;
-  const int n0 = blockIdx.y * BN;
+  const int m_tiles = (M + kProjBM - 1) / kProjBM;
+  const int n_tiles = (Nout + BN - 1) / BN;
+  const int num_tiles = m_tiles * n_tiles;
   const int num_kb = (K + kProjBK - 1) / kProjBK;
 
   if (threadIdx.x == 0) {
@@ -68,11 +95,15 @@ __global__ void __launch_bounds__(128, 1)
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
-    mbar_init(&acc_bar, 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);  // the four epilogue warps
+    }
+    mbar_init(&mma_done, 1);
     abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
+  if (warp == 2) {
     tmem_alloc(&tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -83,35 +114,46 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tacc = tmem_base;
+  const uint32_t tmem = tmem_base;
 
-  if (warp == 0 && lane == 0) {
-    // TMA producer
-    int issued = 0;
-    for (int kb = 0; kb < num_kb; ++kb) {
-      const int s = kb % kProjStages;
-      const uint32_t ph = (kb / kProjStages) & 1;
-      if (kb >= kProjStages && !mbar_wait(&empty_bar[s], ph ^ 1, &abort_flag)) break;
-      mbar_arrive_expect_tx(&full_bar[s], S::kABytes + S::kBBytes);
-      uint8_t* a_dst = a_tiles + s * S::kABytes;
-      uint8_t* b_dst = b_tiles + s * S::kBBytes;
-      if constexpr (kAMN) {
-        for (int c = 0; c < kProjBM / 64; ++c)
-          tma_load_2d(&tm_a, &full_bar[s], a_dst + c * kMnChunk, m0 + 64 * c, kb * kProjBK);
-      } else {
-        tma_load_2d(&tm_a, &full_bar[s], a_dst, kb * kProjBK, m0);
+  if (warp == 0) {
+    if (lane == 0) {
+      // TMA producer; g counts k-blocks over all of this CTA's tiles.
+      int g = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        int mt, nt;
+        proj_tile_coords(tile, m_tiles, n_tiles, mt, nt);
+        const int m0 = mt * kProjBM;
+        const int n0 = nt * BN;
+        for (int kb = 0; kb < num_kb; ++kb, ++g) {
+          const int s = g % kProjStages;
+          const uint32_t ph = (g / kProjStages) & 1;
+          if (g >= kProjStages && !mbar_wait(&empty_bar[s], ph ^ 1, &abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full_bar[s], S::kABytes + S::kBBytes);
+          uint8_t* a_dst = a_tiles + s * S::kABytes;
+          uint8_t* b_dst = b_tiles + s * S::kBBytes;
+          if constexpr (kAMN) {
+            for (int c = 0; c < kProjBM / 64; ++c)
+              tma_load_2d(&tm_a, &full_bar[s], a_dst + c * kMnChunk, m0 + 64 * c, kb * kProjBK);
+          } else {
+            tma_load_2d(&tm_a, &full_bar[s], a_dst, kb * kProjBK, m0);
+          }
+          if constexpr (kBMN) {
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_2d(&tm_b, &full_bar[s], b_dst + c * kMnChunk, n0 + 64 * c, kb * kProjBK);
+          } else {
+            tma_load_2d(&tm_b, &full_bar[s], b_dst, kb * kProjBK, n0);
+          }
+        }
       }
-      if constexpr (kBMN) {
-        for (int c = 0; c < BN / 64; ++c)
-          tma_load_2d(&tm_b, &full_bar[s], b_dst + c * kMnChunk, n0 + 64 * c, kb * kProjBK);
-      } else {
-        tma_load_2d(&tm_b, &full_bar[s], b_dst, kb * kProjBK, n0);
-      }
-      ++issued;
+      // No copy may still be landing in shared memory when the CTA exits.
+      for (int q = g > kProjStages ? g - kProjStages : 0; q < g; ++q)
+        mbar_drain(&full_bar[q % kProjStages], (q / kProjStages) & 1);
     }
-    // No copy may still be landing in shared memory when the CTA exits.
-    for (int kb = issued > kProjStages ? issued - kProjStages : 0; kb < issued; ++kb)
-      mbar_drain(&full_bar[kb % kProjStages], (kb / kProjStages) & 1);
   } else if (warp == 1) {
     // MMA issuer: the whole warp runs the loop (operands stay warp-uniform),
     // lane 0 issues.  Descriptors are built once and advanced by offsets:
@@ -125,70 +167,93 @@ __global__ void __launch_bounds__(128, 1)
                                   : smem_desc(smem_addr(b_tiles), 16, 1024, kSw128);
     constexpr uint32_t kAStep = kAMN ? 16 * 128 : 32;
     constexpr uint32_t kBStep = kBMN ? 16 * 128 : 32;
-    for (int kb = 0; kb < num_kb; ++kb) {
-      const int s = kb % kProjStages;
-      const uint32_t ph = (kb / kProjStages) & 1;
-      if (!mbar_wait(&full_bar[s], ph, &abort_flag)) break;
+    int g = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x, k = 0; tile < num_tiles && ok; tile += gridDim.x, ++k) {
+      const int acc = k & 1;
+      // The epilogue has read this accumulator's previous tile.
+      if (k >= 2 && !mbar_wait(&acc_empty[acc], ((k >> 1) - 1) & 1, &abort_flag)) break;
       tc_fence_after();
-      const uint64_t ad = desc_advance(a_desc0, s * S::kABytes);
-      const uint64_t bd = desc_advance(b_desc0, s * S::kBBytes);
+      const uint32_t tacc = tmem + acc * kAccCols;
+      for (int kb = 0; kb < num_kb; ++kb, ++g) {
+        const int s = g % kProjStages;
+        const uint32_t ph = (g / kProjStages) & 1;
+        if (!mbar_wait(&full_bar[s], ph, &abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t ad = desc_advance(a_desc0, s * S::kABytes);
+        const uint64_t bd = desc_advance(b_desc0, s * S::kBBytes);
 #pragma unroll
-      for (int kk = 0; kk < kProjBK / 16; ++kk)
-        mma_ss_w(tacc, desc_advance(ad, kk * kAStep), desc_advance(bd, kk * kBStep), idesc, (kb | kk) != 0);
-      mma_commit_w(&empty_bar[s]);
+        for (int kk = 0; kk < kProjBK / 16; ++kk)
+          mma_ss_w(tacc, desc_advance(ad, kk * kAStep), desc_advance(bd, kk * kBStep), idesc, (kb | kk) != 0);
+        mma_commit_w(&empty_bar[s]);
+      }
+      if (ok) mma_commit_w(&acc_full[acc]);
     }
-    mma_commit_w(&acc_bar);
-  }
-  __syncwarp();
-
-  // Epilogue: warp w reads TMEM lanes [32w, 32w + 32) = output rows.
-  const bool ok = mbar_wait(&acc_bar, 0, &abort_flag);
-  tc_fence_after();
-  if (ok) {
-    const int row = m0 + warp * 32 + lane;
-    const uint32_t lane_addr = tacc + (static_cast<uint32_t>(warp * 32) << 16);
+    mma_commit_w(&mma_done);
+  } else if (warp >= 4) {
+    // Epilogue: warp w reads TMEM lanes [32 (w - 4), +32) = output rows.
+    const int wq = warp & 3;
+    for (int tile = blockIdx.x, k = 0; tile < num_tiles; tile += gridDim.x, ++k) {
+      const int acc = k & 1;
+      if (!mbar_wait(&acc_full[acc], (k >> 1) & 1, &abort_flag)) break;
+      tc_fence_after();
+      int mt, nt;
+      proj_tile_coords(tile, m_tiles, n_tiles, mt, nt);
+      const int row = mt * kProjBM + wq * 32 + lane;
+      const int n0 = nt * BN;
+      const uint32_t lane_addr = tmem + acc * kAccCols + (static_cast<uint32_t>(wq * 32) << 16);
 #pragma unroll 1
-    for (int c0 = 0; c0 < BN; c0 += 16) {
-      uint32_t r[16];
-      tmem_ld16(lane_addr + c0, r);
-      tmem_wait_ld();
-      const int n = n0 + c0;
-      if (row < M && n < Nout) {
-        float v[16];
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(lane_addr + c0, r);
+        tmem_wait_ld();
+        const int n = n0 + c0;
+        if (row < M && n < Nout) {
+          float v[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]) + (bias != nullptr ? bias[n + i] : 0.f);
-        if constexpr (kOutBf16) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(y) + static_cast<size_t>(row) * Nout + n);
-          dst[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                              pack_bf16x2(v[6], v[7]));
-          dst[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
-                              pack_bf16x2(v[14], v[15]));
-        } else {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(y) + static_cast<size_t>(row) * Nout + n);
+          for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]) + (bias != nullptr ? bias[n + i] : 0.f);
+          if constexpr (kOutBf16) {
+            uint4* dst =
+                reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(y) + static_cast<size_t>(row) * Nout + n);
+            dst[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                                pack_bf16x2(v[6], v[7]));
+            dst[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
+                                pack_bf16x2(v[14], v[15]));
+          } else {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(y) + static_cast<size_t>(row) * Nout + n);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            float4 w = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-            if (accumulate) {
-              const float4 old = dst[i];
-              w.x += old.x;
-              w.y += old.y;
-              w.z += old.z;
-              w.w += old.w;
+            for (int i = 0; i < 4; ++i) {
+              float4 w = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+              if (accumulate) {
+                const float4 old = dst[i];
+                w.x += old.x;
+                w.y += old.y;
+                w.z += old.z;
+                w.w += old.w;
+              }
+              dst[i] = w;
             }
-            dst[i] = w;
           }
         }
       }
+      // Hand the accumulator back to the MMA warp.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
     }
   }
-  // The MMA warp always commits acc_bar, so this returns once every MMA it
-  // issued has finished, also after an abort.
-  if (!ok && threadIdx.x == 0) mbar_drain(&acc_bar, 0);
+
+  // ---- teardown: every MMA the issuer started has finished -----------------
+  __syncwarp();
+  if (threadIdx.x == 32) mbar_drain(&mma_done, 0);
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tacc, kTmemCols);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
