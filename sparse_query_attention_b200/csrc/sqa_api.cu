@@ -807,6 +807,6 @@ const char* sqa_status_string(sqa_status_t status) {
   return "SQA_ERR_UNKNOWN";
 }
 
-const char* sqa_version(void) { return "0.1.0"; }
+const char* sqa_version(void) { return "0.2.0"; }
 
 }  // extern "C"
