@@ -36,6 +36,8 @@ def _bf16(shape, gen, std=1.0):
     (True, True, 256, 256, 16384),    # dW = dY^T X
     (True, True, 16, 256, 4096),      # narrow weight (H_kv * d_head = 16)
     (True, False, 128, 128, 256),
+    (False, True, 20000, 512, 256),   # 314 tiles: several per persistent CTA, ragged last row tile
+    (True, True, 2048, 2048, 512),    # 256 tiles, both operands MN-contiguous
 ])
 def test_gemm_layouts(sqa, a_mn, b_mn, M, N, K):
     g = torch.Generator(device="cuda")
@@ -52,10 +54,10 @@ def test_gemm_layouts(sqa, a_mn, b_mn, M, N, K):
     assert_close(f64(c), projection(A, Bm), "C")
 
 
-def test_gemm_accumulate(sqa):
+@pytest.mark.parametrize("M,N,K", [(512, 256, 64), (40000, 256, 64)])
+def test_gemm_accumulate(sqa, M, N, K):
     g = torch.Generator(device="cuda")
     g.manual_seed(5)
-    M, N, K = 512, 256, 64
     a, b = _bf16((M, K), g), _bf16((K, N), g, 0.05)
     c0 = torch.randn((M, N), generator=g, device="cuda")
     c = c0.clone()
