@@ -330,6 +330,56 @@ def time_windowed(sqa, torch, stream, dev, reps=3):
     return {"config": {"B": 1, "N": N, "d_head": d}, "windows": res}
 
 
+CROSS = {"B": 1, "N_q": 32768, "N_kv": 8192, "d_head": 128}
+
+
+def time_cross(sqa, torch, stream, dev, reps=5):
+    """Cross / memory attention, N_q = 32768 queries against N_kv = 8192 keys
+    of another sequence (B=1, d=128, no mask): forward for MHA, SQA and xSQA
+    on the same kernel, and the SQA backward.  FLOPs 4 * H_q * N_q * N_kv * d
+    forward, 8 * ... backward."""
+    from sqa_inputs import cross_attention_inputs
+
+    c = CROSS
+    B, Nq, Nkv, d = c["B"], c["N_q"], c["N_kv"], c["d_head"]
+    sc = 1 / math.sqrt(d)
+
+    def med(fn):
+        fn()
+        times = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        return statistics.median(times)
+
+    res = {}
+    for name, (hq, hkv) in LONG_VARIANTS.items():
+        x = cross_attention_inputs(B, Nq, Nkv, hq, hkv, d, seed=6, with_dout=name == "SQA", device=dev)
+        o = torch.empty((B, Nq, hq, d), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((B, hq, Nq), dtype=torch.float32, device=dev)
+        BF = sqa.SQA_DT_BF16
+        ms = med(lambda: sqa.sqa_attn_fwd_cross(x["q"], x["k"], x["v"], o, BF, lse, B, Nq, Nkv, hq, hkv, d, sc,
+                                                stream=stream))
+        flops = 4 * B * hq * Nq * Nkv * d
+        res[name] = {"H_q": hq, "H_kv": hkv, "fwd_ms": ms, "fwd_tflops": flops / ms / 1e9}
+        if name == "SQA":
+            dq, dk, dv = (torch.empty(t.shape, dtype=torch.bfloat16, device=dev) for t in (x["q"], x["k"], x["v"]))
+            wsb = sqa.sqa_attn_bwd_workspace_size(B, Nq, hq, hkv, d)
+            ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+            bms = med(lambda: sqa.sqa_attn_bwd_cross(x["q"], x["k"], x["v"], o, BF, x["do"], lse, dq, dk, dv, BF, B,
+                                                     Nq, Nkv, hq, hkv, d, sc, ws, wsb, stream=stream))
+            res[name].update({"bwd_ms": bms, "bwd_tflops": 2 * flops / bms / 1e9})
+        del x, o, lse
+    for name in res:
+        res[name]["fwd_speedup_vs_mha"] = res["MHA"]["fwd_ms"] / res[name]["fwd_ms"]
+    sqa.sqa_device_status(stream)
+    return {"config": dict(c), "variants": res}
+
+
 DECODE = {"B": 16, "L": 32768, "n_new": 1, "d_head": 128}
 DECODE_VARIANTS = {"MHA": (16, 16), "GQA": (16, 4), "SQA": (8, 4), "xSQA": (4, 4), "xSMQA": (4, 1)}
 
@@ -680,6 +730,7 @@ def run_sqa(args):
     long_seq = time_long_sequences(sqa, torch, stream, dev)
     windowed = time_windowed(sqa, torch, stream, dev)
     decode = time_decode(sqa, torch, stream, dev)
+    cross = time_cross(sqa, torch, stream, dev)
 
     peak, peak_kind = load_peaks()
     achieved = flops_step / (statistics.mean(per_launch_ms) / 1e3) / 1e12
@@ -704,6 +755,7 @@ def run_sqa(args):
         "long_sequences": long_seq,
         "windowed": windowed,
         "decode": decode,
+        "cross": cross,
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
