@@ -143,3 +143,10 @@ def test_fwd_deterministic(sqa):
     o1, l1 = run_fwd(sqa, x["q"], x["k"], x["v"], True)
     o2, l2 = run_fwd(sqa, x["q"], x["k"], x["v"], True)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("H_q,H_kv,causal", [(32, 1, True), (64, 1, False), (128, 1, True), (128, 2, False)])
+def test_fwd_wide_groups(sqa, H_q, H_kv, causal):
+    """G = 32 .. 128 query heads per KV head: a 128-row tile packs 128 / G
+    tokens (down to one token of 128 heads), the limit of the head packing."""
+    _check_fwd(sqa, 1, 200, H_q, H_kv, 64, causal, seed=200 + H_q)
