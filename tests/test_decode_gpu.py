@@ -96,3 +96,18 @@ def test_decode_bad_length_is_reported(sqa):
     sqa.sqa_device_status()  # cleared
     ro, _ = attention_decode(f64(q), f64(kc), f64(vc), np.asarray([L_max, 10]), 1 / math.sqrt(d))
     assert_close(f64(o), ro, "O (clamped length)")
+
+
+def test_decode_bench_configuration(sqa):
+    """The benchmark's decode step exactly: B=16 sequences with 32768 cached
+    tokens each, SQA (8, 4), d=128, one new token, bf16 output (18 chunks of
+    1856 keys per sequence and KV head, merged by the combine pass)."""
+    B, n_new, H_q, H_kv, d, L_max = 16, 1, 8, 4, 128, 32768
+    assert sqa.sqa_attn_decode_workspace_size(B, n_new, H_q, H_kv, d, L_max) > 0
+    q, kc, vc = _inputs(B, n_new, H_q, H_kv, d, L_max, seed=5)
+    o, lse = _decode(sqa, q, kc, vc, [L_max] * B, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    sqa.sqa_device_status()
+    ro, rl = attention_decode(f64(q), f64(kc), f64(vc), np.full(B, L_max), 1 / math.sqrt(d))
+    assert_close(f64(o), ro, "O")
+    assert_close(f64(lse), rl, "LSE")
