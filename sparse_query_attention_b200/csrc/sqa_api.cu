@@ -340,7 +340,7 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
 
   // 1. D and LSE in log2 units.
   const size_t prep_rows = static_cast<size_t>(B) * H_q * n_pad;
-  sqa::bwd_prep_kernel<D><<<static_cast<unsigned>((prep_rows * 32 + 255) / 256), 256, 0, st>>>(
+  sqa::bwd_prep_kernel<D><<<static_cast<unsigned>((prep_rows * (D / 8) + 255) / 256), 256, 0, st>>>(
       o, o_bf16, static_cast<const __nv_bfloat16*>(dout), lse, dsum, lse2, B, N, H_q, n_pad);
   if (cudaGetLastError() != cudaSuccess) return SQA_ERR_CUDA;
 

@@ -39,33 +39,55 @@ namespace sqa {
 // Preprocess: D[b,h,t] = sum_c dO[b,t,h,c] O[b,t,h,c]; L2[b,h,t] = LSE * log2 e,
 // both stored negated.  Workspace rows are padded to n_pad tokens (multiple of
 // 128) with zeros.
-// One warp per (b, h, t) of the padded space.
+// HBM-bound: kLanes = D / 8 lanes per row, each reading 8 consecutive
+// elements of O (fp32: two 16-byte loads; bf16: one) and of dO (one 16-byte
+// load), so a warp covers 256 / D rows with fully used 16-byte accesses.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void bwd_prep_kernel(const void* __restrict__ o, int o_bf16, const __nv_bfloat16* __restrict__ dout,
                                 const float* __restrict__ lse, float* __restrict__ dsum, float* __restrict__ lse2,
                                 int B, int N, int H_q, int n_pad) {
-  const size_t idx = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
-  const int lane = threadIdx.x & 31;
+  constexpr int kLanes = D / 8;  // 2 .. 16 lanes per row
+  const size_t gtid = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const size_t idx = gtid / kLanes;  // row of the padded [B, H_q, n_pad] space
+  const int sub = static_cast<int>(gtid % kLanes);
   const size_t total = static_cast<size_t>(B) * H_q * n_pad;
-  if (idx >= total) return;
-  const int t = static_cast<int>(idx % n_pad);
-  const size_t bh = idx / n_pad;
+  const bool in = idx < total;
+  const int t = in ? static_cast<int>(idx % n_pad) : 0;
+  const size_t bh = in ? idx / n_pad : 0;
   const int h = static_cast<int>(bh % H_q);
   const int b = static_cast<int>(bh / H_q);
   float acc = 0.f, l2 = 0.f;
-  if (t < N) {
-    const size_t row = ((static_cast<size_t>(b) * N + t) * H_q + h) * D;
-    for (int c = lane; c < D; c += 32) {
-      const float ov = o_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(o)[row + c])
-                              : static_cast<const float*>(o)[row + c];
-      acc = fmaf(ov, __bfloat162float(dout[row + c]), acc);
+  if (in && t < N) {
+    const size_t base = ((static_cast<size_t>(b) * N + t) * H_q + h) * D + sub * 8;
+    const uint4 g = *reinterpret_cast<const uint4*>(dout + base);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
+    float ov[8];
+    if (o_bf16) {
+      const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(o) + base);
+      const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __bfloat1622float2(u2[k]);
+        ov[2 * k] = f.x;
+        ov[2 * k + 1] = f.y;
+      }
+    } else {
+      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(o) + base);
+      const float4 a = src[0], c = src[1];
+      ov[0] = a.x, ov[1] = a.y, ov[2] = a.z, ov[3] = a.w, ov[4] = c.x, ov[5] = c.y, ov[6] = c.z, ov[7] = c.w;
     }
 #pragma unroll
-    for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __bfloat1622float2(g2[k]);
+      acc = fmaf(ov[2 * k], f.x, acc);
+      acc = fmaf(ov[2 * k + 1], f.y, acc);
+    }
     l2 = lse[bh * N + t] * 1.4426950408889634f;
   }
-  if (lane == 0) {  // stored negated: the kernels add them in packed FFMA/FADD
+#pragma unroll
+  for (int s = kLanes / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  if (in && sub == 0) {  // stored negated: the kernels add them in packed FFMA/FADD
     dsum[idx] = -acc;
     lse2[idx] = -l2;
   }
