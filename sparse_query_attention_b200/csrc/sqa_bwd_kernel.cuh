@@ -146,7 +146,7 @@ struct BwdParams {
   int g, log2g, n_sub, n_tblk;  // packing of the dQ kernel
   int masked;                   // band mask active (causal or sliding window)
   int win_l, win_r;             // band: t - win_l <= u <= t + win_r (both <= N)
-  int longest_first;            // dQ: schedule token blocks from the last one
+  int longest_first;            // causal: hand out the longest tiles first over the whole grid
   float scale;
   float scale_log2;
 };
@@ -231,9 +231,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   const int warp = warp_id_uniform();
   const int lane = threadIdx.x & 31;
-  const int kt = blockIdx.x;  // key tile
-  const int j = blockIdx.y;
-  const int b = blockIdx.z;
+  // Causal: key tile 0 sees every query, so ascending tiles are longest first.
+  const BlockUnit u = block_unit(p.longest_first);
+  const int kt = u.x;  // key tile
+  const int j = u.y;
+  const int b = u.z;
   const int key0 = kt * 128;
   // Queries that can see a key of this tile: t in [key0 - win_r,
   // key0 + 127 + win_l] within [0, N); streamed as 64-token sub-tiles.
@@ -622,10 +624,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = warp_id_uniform();
   const int lane = threadIdx.x & 31;
   const int T = 128 >> p.log2g;
-  const int tblk = p.longest_first ? (p.n_tblk - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
-  const int j = blockIdx.y / p.n_sub;
-  const int sub = blockIdx.y % p.n_sub;
-  const int b = blockIdx.z;
+  const BlockUnit u = block_unit(p.longest_first);
+  const int tblk = p.longest_first ? (p.n_tblk - 1 - u.x) : u.x;
+  const int j = u.y / p.n_sub;
+  const int sub = u.y % p.n_sub;
+  const int b = u.z;
   const int h0 = j * p.G + sub * p.g;
   const int t0 = tblk * T;
   const int last_tok = min(t0 + T, p.N) - 1;

@@ -102,10 +102,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   // ---- work unit -----------------------------------------------------------
   const int T = 128 >> p.log2g;  // tokens per tile
-  const int tblk = p.longest_first ? (p.n_tblk - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
-  const int j = blockIdx.y / p.n_sub;
-  const int sub = blockIdx.y % p.n_sub;
-  const int b = blockIdx.z;
+  const BlockUnit u = block_unit(p.longest_first);
+  const int tblk = p.longest_first ? (p.n_tblk - 1 - u.x) : u.x;
+  const int j = u.y / p.n_sub;
+  const int sub = u.y % p.n_sub;
+  const int b = u.z;
   const int h0 = j * p.G + sub * p.g;
   const int t0 = tblk * 2 * T;  // tile 0 tokens [t0, t0+T), tile 1 [t0+T, t0+2T)
   // KV tiles [kv_lo[t], kv_hi[t]) hold every key a row of query tile t can

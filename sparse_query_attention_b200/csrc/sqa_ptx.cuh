@@ -458,6 +458,23 @@ __device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, fl
   y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
+// Work unit (x, y, z) of this block.  With x_major the grid's x index
+// orders the units by length (x = 0 the longest): the hardware hands blocks
+// out in linear order, x fastest, so the linear index is re-read with x
+// slowest, and every (y, z) pair of one x is handed out before the next x --
+// longest first across the whole grid, not only within each (y, z) row.
+struct BlockUnit {
+  int x, y, z;
+};
+__device__ __forceinline__ BlockUnit block_unit(bool x_major) {
+  if (!x_major) return {static_cast<int>(blockIdx.x), static_cast<int>(blockIdx.y), static_cast<int>(blockIdx.z)};
+  const unsigned long long yz = static_cast<unsigned long long>(gridDim.y) * gridDim.z;
+  const unsigned long long lin =
+      blockIdx.x + static_cast<unsigned long long>(gridDim.x) * (blockIdx.y + static_cast<unsigned long long>(gridDim.y) * blockIdx.z);
+  const unsigned long long r = lin % yz;
+  return {static_cast<int>(lin / yz), static_cast<int>(r % gridDim.y), static_cast<int>(r / gridDim.y)};
+}
+
 // Per-warpgroup register reallocation.  The block launches with
 // threads x (registers per thread); the counts requested by all warpgroups
 // must add up to no more than that pool.

@@ -82,6 +82,28 @@ def test_fwd_large_scores_and_custom_scale(sqa, causal):
     _check_fwd(sqa, 1, 640, 4, 4, 64, causal, seed=5, scale=1.0, mult=1.25)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_fwd_running_max_jumps(sqa, causal, d):
+    """Key blocks whose scores jump by ~8-20 and by ~30-60 log2 units over
+    the running max of the blocks before them: the first kind is kept
+    against the stale max and moved at the next block, the second is
+    recomputed in two passes from the scores."""
+    N = 1024
+    x = attention_inputs(1, N, 4, 2, d, seed=31 + d, device="cuda")
+    k = x["k"].float()
+    k[:, 256:384] *= 4.0
+    k[:, 640:768] *= 12.0
+    k[:, 900:1000] *= 0.25
+    x["k"] = k.to(torch.bfloat16)
+    o, lse = run_fwd(sqa, x["q"], x["k"], x["v"], causal)
+    torch.cuda.synchronize()
+    sqa.sqa_device_status()
+    o_ref, lse_ref = _oracle_fwd(x, causal)
+    assert_close(f64(o), o_ref, "O")
+    assert_close(f64(lse), lse_ref, "LSE")
+
+
 @pytest.mark.parametrize("H_q,H_kv,causal", [(6, 2, True), (12, 4, False), (6, 1, True), (24, 8, False)])
 def test_fwd_group_not_power_of_two(sqa, H_q, H_kv, causal):
     """G = 3 or 6: the tile packs the largest power of two dividing G and a
