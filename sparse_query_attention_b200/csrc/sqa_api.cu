@@ -13,6 +13,7 @@
 #include "sqa_bwd_kernel.cuh"
 #include "sqa_decode_kernel.cuh"
 #include "sqa_fwd_kernel.cuh"
+#include "sqa_fwd_quad_kernel.cuh"
 #include "sqa_proj_kernel.cuh"
 #include "sqa_ptx.cuh"
 
@@ -222,11 +223,20 @@ sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* ou
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const long long gy = static_cast<long long>(H_kv) * p.n_sub;
   if (gy > 65535 || B > 65535) return SQA_ERR_UNSUPPORTED;
-  auto kern = sqa::sqa_fwd_kernel<D>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
-    return SQA_ERR_CUDA;
   dim3 grid(p.n_tblk, static_cast<unsigned>(gy), B);
-  kern<<<grid, sqa::kFwdThreads, C::kSmemBytes, st>>>(mq, mk, mv, p);
+  if constexpr (D <= 64) {
+    // Four virtual tiles (two key halves per query tile): see sqa_fwd_quad_kernel.cuh.
+    auto kern = sqa::sqa_fwd_quad_kernel<D>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sqa::QuadCfg<D>::kSmemBytes) !=
+        cudaSuccess)
+      return SQA_ERR_CUDA;
+    kern<<<grid, sqa::kQuadThreads, sqa::QuadCfg<D>::kSmemBytes, st>>>(mq, mk, mv, p);
+  } else {
+    auto kern = sqa::sqa_fwd_kernel<D>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+      return SQA_ERR_CUDA;
+    kern<<<grid, sqa::kFwdThreads, C::kSmemBytes, st>>>(mq, mk, mv, p);
+  }
   return launch_status();
 }
 
