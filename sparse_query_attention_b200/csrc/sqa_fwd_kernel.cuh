@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (!mbar_wait(&p_ready[0][1], i & 1, &abort_flag)) break;
         tc_fence_after();
         issue_pv(0, vs, true, 4);
-        mma_commit_w(&o_done[0]);
+        if (!more) mma_commit_w(&o_done[0]);  // the epilogue's signal; S(i+1) carries it otherwise
         if (more) {
           issue_s(0, ks);
           mma_commit_w(&s_full[0]);
@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (!mbar_wait(&p_ready[1][1], i & 1, &abort_flag)) break;
         tc_fence_after();
         issue_pv(1, vs, true, 4);
-        mma_commit_w(&o_done[1]);
+        if (!more) mma_commit_w(&o_done[1]);
         mma_commit_w(&slot_empty[vs]);
         if (more) {
           issue_s(1, ks);
@@ -360,12 +360,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // the stale max, which bounds P by 2^8.
       const bool grow = m_new > m_used + kRescaleThreshold || (m_used == -INFINITY && m_new != -INFINITY);
       if (__any_sync(0xffffffffu, grow && i > 0 && m_used != -INFINITY)) {
-        // O holds sum over steps < i; it is final once PV(i-1) completed.
-        if (!mbar_wait(&o_done[t], (i - 1) & 1, &abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+        // O holds the sum over steps < i, and it is final: PV(i-1) was
+        // issued before S(i), and the commit that signalled S(i) tracks
+        // every earlier MMA of the issuing thread.
         const float f = (grow && m_used != -INFINITY) ? ex2_approx(m_used - m_new) : 1.f;
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 16) {
@@ -421,7 +418,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
     }
     // Epilogue: O / l and LSE once the last PV of this tile has landed.
-    if (ok) ok = mbar_wait(&o_done[t], (my_steps - 1) & 1, &abort_flag);
+    if (ok) ok = mbar_wait(&o_done[t], 0, &abort_flag);  // committed once, after the last PV
     if (ok) {
       tc_fence_after();
       const bool valid = tok < p.N;

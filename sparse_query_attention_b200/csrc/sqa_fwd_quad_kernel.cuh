@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(kQuadThreads, 1)
         }
         tc_fence_after();
         issue_pv(v, vs, i > 0);
-        mma_commit_w(&o_done[v]);
+        if (!more) mma_commit_w(&o_done[v]);  // the epilogue's signal; S(i+1) carries it otherwise
         if (more) {
           issue_s(v, ks);
           mma_commit_w(&s_full[v]);
@@ -305,12 +305,9 @@ __global__ void __launch_bounds__(kQuadThreads, 1)
       // (or on the first finite max), which bounds P by 2^8.
       const bool grow = m_new > m_used + kRescaleThreshold || (m_used == -INFINITY && m_new != -INFINITY);
       if (__any_sync(0xffffffffu, grow && i > 0 && m_used != -INFINITY)) {
-        // O_v holds the sum over steps < i; it is final once PV(i-1) completed.
-        if (!mbar_wait(&o_done[v], (i - 1) & 1, &abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+        // O_v holds the sum over steps < i, and it is final: PV(i-1) was
+        // issued before S(i), and the commit that signalled S(i) tracks
+        // every earlier MMA of the issuing thread.
         const float f = (grow && m_used != -INFINITY) ? ex2_approx(m_used - m_new) : 1.f;
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 16) {
@@ -362,8 +359,8 @@ __global__ void __launch_bounds__(kQuadThreads, 1)
     // columns [0, d/2) and the LSE, half 1 columns [d/2, d) (half 0 alone at
     // d = 16).  Every thread of the query tile reaches the named barrier,
     // also after a timeout, so none is left waiting there.
-    if (ok) ok = mbar_wait(&o_done[v], (n_steps - 1) & 1, &abort_flag);
-    if (ok) ok = mbar_wait(&o_done[v ^ 2], (n_steps - 1) & 1, &abort_flag);
+    if (ok) ok = mbar_wait(&o_done[v], 0, &abort_flag);  // committed once, after the last PV
+    if (ok) ok = mbar_wait(&o_done[v ^ 2], 0, &abort_flag);
     merge_m[v][r] = m_used;
     merge_l[v][r] = l_sum;
     named_bar_sync(1 + qt, 256);
