@@ -68,6 +68,28 @@ def weak_scaling_rate(world, units_per_rank_step, steps, max_ms):
     return world * units_per_rank_step * steps / (max_ms / 1e3)
 
 
+def device_times(torch, stream, fns, reps, before=None):
+    """Device time of each call in `fns`, per repetition: CUDA events on the
+    launching stream around every call.  All repetitions are enqueued ahead
+    and the host synchronises once at the end, so the host-side launch path
+    overlaps the device work of earlier repetitions instead of landing inside
+    a timed interval (a per-repetition synchronise leaves the device idle
+    while the host launches).  `before` (an L2 flush) runs ahead of each
+    repetition, outside its intervals.  Returns one list of ms per call."""
+    marks = []
+    for _ in range(reps):
+        if before is not None:
+            before()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
+        ev[0].record(stream)
+        for k, fn in enumerate(fns):
+            fn()
+            ev[k + 1].record(stream)
+        marks.append(ev)
+    marks[-1][-1].synchronize()
+    return [[ev[k].elapsed_time(ev[k + 1]) for ev in marks] for k in range(len(fns))]
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -234,17 +256,12 @@ def time_long_sequences(sqa, torch, stream, dev, reps=3):
         for name, (hq, hkv) in LONG_VARIANTS.items():
             x = attention_inputs(1, N, hq, hkv, d, seed=3, device=dev)
             o = torch.empty((1, N, hq * d), dtype=torch.float32, device=dev)
-            sqa.sqa_attn_fwd(x["q"], x["k"], x["v"], o, 1, N, hq, hkv, d, False, 1 / math.sqrt(d), stream=stream)
-            times = []
-            for _ in range(reps):
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
+            def fwd():
                 sqa.sqa_attn_fwd(x["q"], x["k"], x["v"], o, 1, N, hq, hkv, d, False, 1 / math.sqrt(d),
                                  stream=stream)
-                b.record(stream)
-                b.synchronize()
-                times.append(a.elapsed_time(b))
-            ms = statistics.median(times)
+
+            fwd()
+            ms = statistics.median(device_times(torch, stream, [fwd], reps)[0])
             per[name] = {"H_q": hq, "H_kv": hkv, "ms": ms,
                          "tflops": attn_fwd_flops(1, N, hq, d, False) / ms / 1e9, "tokens_per_s": N / (ms / 1e3)}
             del x, o
@@ -282,15 +299,7 @@ def time_windowed(sqa, torch, stream, dev, reps=3):
 
     def med(fn):
         fn()
-        times = []
-        for _ in range(reps):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            fn()
-            b.record(stream)
-            b.synchronize()
-            times.append(a.elapsed_time(b))
-        return statistics.median(times)
+        return statistics.median(device_times(torch, stream, [fn], reps)[0])
 
     res = {}
     for wname, (left, right) in c["windows"].items():
@@ -346,15 +355,7 @@ def time_cross(sqa, torch, stream, dev, reps=5):
 
     def med(fn):
         fn()
-        times = []
-        for _ in range(reps):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            fn()
-            b.record(stream)
-            b.synchronize()
-            times.append(a.elapsed_time(b))
-        return statistics.median(times)
+        return statistics.median(device_times(torch, stream, [fn], reps)[0])
 
     res = {}
     for name, (hq, hkv) in LONG_VARIANTS.items():
@@ -396,8 +397,9 @@ def time_decode(sqa, torch, stream, dev, reps=10):
     """One decode step (n_new = 1) for B = 16 sequences with 32768 cached
     tokens, d = 128, per head-count variant.  HBM-bound: algorithmic bytes
     are the K and V cache (2 * B * L * H_kv * d bf16) plus Q and O; the cache
-    is larger than L2 at every variant but xSMQA (128 MiB), so no flush is
-    added.  Reported against the measured copy bandwidth."""
+    (256 MiB at xSMQA's single KV head, 4 GiB at MHA) is larger than the L2 at
+    every variant, so no flush is added.  Steps run back to back, as decode
+    steps do in serving.  Reported against the measured copy bandwidth."""
     c = DECODE
     B, L, n_new, d = c["B"], c["L"], c["n_new"], c["d_head"]
     peak, kind = load_hbm_peak()
@@ -419,15 +421,7 @@ def time_decode(sqa, torch, stream, dev, reps=10):
 
         for _ in range(3):
             step()
-        times = []
-        for _ in range(reps):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            step()
-            b.record(stream)
-            b.synchronize()
-            times.append(a.elapsed_time(b))
-        ms = statistics.median(times)
+        ms = statistics.median(device_times(torch, stream, [step], reps)[0])
         nbytes = 2 * B * L * hkv * d * 2 + 2 * B * n_new * hq * d * 2
         res[name] = {"H_q": hq, "H_kv": hkv, "ms": ms, "gbs": nbytes / ms / 1e6, "frac_hbm": nbytes / ms / 1e6 / peak,
                      "tokens_per_s": B * n_new / (ms / 1e3)}
@@ -492,16 +486,7 @@ def time_decoder_layer(sqa, torch, stream, flush, dev, reps=5):
         def timed(fn):
             for _ in range(3):
                 fn()
-            times = []
-            for _ in range(reps):
-                flush.fill_(3)
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                fn()
-                b.record(stream)
-                b.synchronize()
-                times.append(a.elapsed_time(b))
-            return statistics.median(times)
+            return statistics.median(device_times(torch, stream, [fn], reps, before=lambda: flush.fill_(3))[0])
 
         def step():
             layer()
@@ -551,18 +536,7 @@ def time_training_step(sqa, torch, stream, flush, dev, reps=5):
     for _ in range(3):
         fwd()
         bwd()
-    tf, tb = [], []
-    for _ in range(reps):
-        flush.fill_(2)
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-        e[0].record(stream)
-        fwd()
-        e[1].record(stream)
-        bwd()
-        e[2].record(stream)
-        e[2].synchronize()
-        tf.append(e[0].elapsed_time(e[1]))
-        tb.append(e[1].elapsed_time(e[2]))
+    tf, tb = device_times(torch, stream, [fwd, bwd], reps, before=lambda: flush.fill_(2))
     sqa.sqa_device_status(stream)
     ms_f, ms_b = statistics.median(tf), statistics.median(tb)
     f_fwd = attn_fwd_flops(B, N, H_q, d, True)
@@ -708,15 +682,8 @@ def run_sqa(args):
         ov = torch.empty((B, N, vq * d), dtype=torch.float32, device=dev)
         for _ in range(2):
             step(xv["q"], xv["k"], xv["v"], ov, vq, vkv)
-        times = []
-        for _ in range(5):
-            flush.fill_(1)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            step(xv["q"], xv["k"], xv["v"], ov, vq, vkv)
-            b.record(stream)
-            b.synchronize()
-            times.append(a.elapsed_time(b))
+        times = device_times(torch, stream, [lambda: step(xv["q"], xv["k"], xv["v"], ov, vq, vkv)], 5,
+                             before=lambda: flush.fill_(1))[0]
         ms = statistics.median(times)
         variants[name] = {"H_q": vq, "H_kv": vkv, "ms": ms,
                           "tflops": attn_fwd_flops(B, N, vq, d, w["causal"]) / (ms / 1e3) / 1e12}

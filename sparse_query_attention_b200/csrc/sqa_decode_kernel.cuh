@@ -171,6 +171,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             tma_load_4d(m, &slot_full[s], dst + c * C::kKvChunkBytes, c * C::kRowElems, j, kstart + i * C::kBK, b);
         }
       }
+      // Every load of this CTA is issued: the combine pass may be scheduled
+      // once all CTAs are here (it waits for this grid to finish anyway).
+      grid_launch_dependents();
       mbar_drain(&q_full, 0);
       for (int l = max(0, load - C::kSlots); l < load; ++l) mbar_drain(&slot_full[l % C::kSlots], (l / C::kSlots) & 1);
     }
@@ -376,56 +379,83 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 }
 
 // ---------------------------------------------------------------------------
-// Merge of the per-chunk results: one warp per (b, token, head) row; lane l
-// holds columns [l * k, (l + 1) * k), k = max(1, D / 32) (at D = 16 lanes
-// 16-31 idle).
+// Merge of the per-chunk results: one 256-thread block per (b, token, head)
+// row.  Its eight warps take the chunks in turn (warp w: chunks w, w + 8, ...),
+// lane l holding columns [l * k, (l + 1) * k), k = max(1, D / 32) (at D = 16
+// lanes 16-31 idle), so a row's chunks are read eight at a time rather than
+// one after another; the warps' partial sums meet in shared memory.
 //   M = max_s L_s,  w_s = 2^(L_s - M),  O = sum_s w_s O_s / sum_s w_s,
 //   LSE = (M + log2 sum_s w_s) ln 2
 // over the chunks s that start inside sequence b.
 // ---------------------------------------------------------------------------
+constexpr int kCombineWarps = 8;
+
 template <int D>
-__global__ void decode_combine_kernel(const DecParams p) {
+__global__ void __launch_bounds__(kCombineWarps * 32) decode_combine_kernel(const DecParams p) {
   constexpr int kPer = D >= 32 ? D / 32 : 1;
+  __shared__ float sm_acc[kCombineWarps][D];
+  __shared__ float sm_w[kCombineWarps];
   const size_t n_rows = static_cast<size_t>(p.B) * p.n_new * p.H_q;
-  const size_t row = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+  const size_t row = blockIdx.x;  // grid = n_rows
+  grid_dependency_wait();          // the partial results of the decode grid are complete
+  const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  if (row >= n_rows) return;
   const int head = static_cast<int>(row % p.H_q);
   const int tok = static_cast<int>((row / p.H_q) % p.n_new);
   const int b = static_cast<int>(row / (static_cast<size_t>(p.H_q) * p.n_new));
   const int len = decode_len(p, b, false);
   const int n_used = (len + p.chunk - 1) / p.chunk;
+  // Every warp forms the same M (same values, same order).
   float M = -INFINITY;
-  for (int s = 0; s < n_used; ++s) M = fmaxf(M, p.part_l[static_cast<size_t>(s) * n_rows + row]);
+  for (int s = lane; s < n_used; s += 32) M = fmaxf(M, p.part_l[static_cast<size_t>(s) * n_rows + row]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float acc[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
   float wsum = 0.f;
   const bool on = lane * kPer < D;
-  for (int s = 0; s < n_used; ++s) {
+#pragma unroll 2
+  for (int s = warp; s < n_used; s += kCombineWarps) {
     const float ls = p.part_l[static_cast<size_t>(s) * n_rows + row];
     const float w = ls == -INFINITY ? 0.f : exp2f(ls - M);
     wsum += w;
     if (on) {
       const float* src = p.part_o + (static_cast<size_t>(s) * n_rows + row) * D + lane * kPer;
+      if constexpr (kPer == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(src);
+        acc[0] = fmaf(w, v.x, acc[0]);
+        acc[1] = fmaf(w, v.y, acc[1]);
+        acc[2] = fmaf(w, v.z, acc[2]);
+        acc[3] = fmaf(w, v.w, acc[3]);
+      } else {
 #pragma unroll
-      for (int e = 0; e < kPer; ++e) acc[e] = fmaf(w, src[e], acc[e]);
+        for (int e = 0; e < kPer; ++e) acc[e] = fmaf(w, src[e], acc[e]);
+      }
     }
   }
-  const float inv = 1.f / wsum;
   if (on) {
-    if (p.out_bf16) {
-      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + row * D + lane * kPer;
 #pragma unroll
-      for (int e = 0; e < kPer; ++e) dst[e] = __float2bfloat16_rn(acc[e] * inv);
-    } else {
-      float* dst = static_cast<float*>(p.out) + row * D + lane * kPer;
-#pragma unroll
-      for (int e = 0; e < kPer; ++e) dst[e] = acc[e] * inv;
-    }
+    for (int e = 0; e < kPer; ++e) sm_acc[warp][lane * kPer + e] = acc[e];
   }
-  if (lane == 0 && p.lse != nullptr)
-    p.lse[(static_cast<size_t>(b) * p.H_q + head) * p.n_new + tok] = (M + __log2f(wsum)) * 0.69314718055994531f;
+  if (lane == 0) sm_w[warp] = wsum;
+  __syncthreads();
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    float a = 0.f, wt = 0.f;
+#pragma unroll
+    for (int g = 0; g < kCombineWarps; ++g) {
+      a += sm_acc[g][c];
+      wt += sm_w[g];
+    }
+    const float v = a / wt;
+    if (p.out_bf16)
+      static_cast<__nv_bfloat16*>(p.out)[row * D + c] = __float2bfloat16_rn(v);
+    else
+      static_cast<float*>(p.out)[row * D + c] = v;
+    if (c == 0 && p.lse != nullptr)
+      p.lse[(static_cast<size_t>(b) * p.H_q + head) * p.n_new + tok] = (M + __log2f(wt)) * 0.69314718055994531f;
+  }
 }
 
 }  // namespace sqa

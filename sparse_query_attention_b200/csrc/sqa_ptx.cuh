@@ -475,6 +475,16 @@ __device__ __forceinline__ BlockUnit block_unit(bool x_major) {
   return {static_cast<int>(lin / yz), static_cast<int>(r % gridDim.y), static_cast<int>(r / gridDim.y)};
 }
 
+// Programmatic dependent launch.  A grid launched after this one on the same
+// stream with programmatic stream serialization may be scheduled once every
+// CTA of this grid has called grid_launch_dependents (or exited); it must
+// call grid_dependency_wait, which returns when this grid has completed and
+// its memory writes are visible, before it reads anything this grid wrote.
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Per-warpgroup register reallocation.  The block launches with
 // threads x (registers per thread); the counts requested by all warpgroups
 // must add up to no more than that pool.
