@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "sqa.h"
 #include "sqa_bwd_kernel.cuh"
@@ -60,6 +61,28 @@ inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 sqa_status_t launch_status() {
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
+}
+
+// Every kernel of the library is launched with programmatic stream
+// serialization: it may be scheduled while the previous kernel on the stream
+// finishes, runs its set-up (barriers, TMEM allocation, descriptor
+// prefetch) meanwhile, and waits in grid_dependency_wait for that kernel to
+// complete before it touches global memory.  Stream order is kept for
+// everything the kernels read and write.
+template <typename... KArgs, typename... Args>
+sqa_status_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                      Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
 }
 
 bool supported_d(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
@@ -230,14 +253,13 @@ sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* ou
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sqa::QuadCfg<D>::kSmemBytes) !=
         cudaSuccess)
       return SQA_ERR_CUDA;
-    kern<<<grid, sqa::kQuadThreads, sqa::QuadCfg<D>::kSmemBytes, st>>>(mq, mk, mv, p);
+    return launch_k(kern, grid, dim3(sqa::kQuadThreads), sqa::QuadCfg<D>::kSmemBytes, st, mq, mk, mv, p);
   } else {
     auto kern = sqa::sqa_fwd_kernel<D>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
       return SQA_ERR_CUDA;
-    kern<<<grid, sqa::kFwdThreads, C::kSmemBytes, st>>>(mq, mk, mv, p);
+    return launch_k(kern, grid, dim3(sqa::kFwdThreads), C::kSmemBytes, st, mq, mk, mv, p);
   }
-  return launch_status();
 }
 
 sqa_status_t attn_fwd_impl(const void* q, const void* k, const void* v, void* out, sqa_dtype_t out_dtype, float* lse,
@@ -350,9 +372,10 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
 
   // 1. D and LSE in log2 units.
   const size_t prep_rows = static_cast<size_t>(B) * H_q * n_pad;
-  sqa::bwd_prep_kernel<D><<<static_cast<unsigned>((prep_rows * (D / 8) + 255) / 256), 256, 0, st>>>(
-      o, o_bf16, static_cast<const __nv_bfloat16*>(dout), lse, dsum, lse2, B, N, H_q, n_pad);
-  if (cudaGetLastError() != cudaSuccess) return SQA_ERR_CUDA;
+  sqa_status_t s = launch_k(sqa::bwd_prep_kernel<D>, dim3(static_cast<unsigned>((prep_rows * (D / 8) + 255) / 256)),
+                            dim3(256), 0, st, o, o_bf16, static_cast<const __nv_bfloat16*>(dout), lse, dsum, lse2, B,
+                            N, H_q, n_pad);
+  if (s != SQA_OK) return s;
 
   // 2. dK, dV (KV-outer).  The statistics ride in the score MMAs unless
   // 1 / (scale log2 e) is out of range (a zero or near-zero scale).
@@ -363,8 +386,8 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return SQA_ERR_CUDA;
     dim3 grid((Nkv + 127) / 128, H_kv, B);
-    kern<<<grid, sqa::kBwdThreads, smem, st>>>(m_k128, m_v128, m_q64, m_do64, m_l2, m_ds, p);
-    if (cudaGetLastError() != cudaSuccess) return SQA_ERR_CUDA;
+    s = launch_k(kern, grid, dim3(sqa::kBwdThreads), smem, st, m_k128, m_v128, m_q64, m_do64, m_l2, m_ds, p);
+    if (s != SQA_OK) return s;
   }
   // 3. dQ (Q-outer).
   {
@@ -373,9 +396,8 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return SQA_ERR_CUDA;
     dim3 grid(p.n_tblk, static_cast<unsigned>(gy), B);
-    kern<<<grid, sqa::kBwdThreads, smem, st>>>(m_qp, m_dop, m_k64, m_v64, p);
+    return launch_k(kern, grid, dim3(sqa::kBwdThreads), smem, st, m_qp, m_dop, m_k64, m_v64, p);
   }
-  return launch_status();
 }
 
 template <int D>
@@ -425,8 +447,7 @@ sqa_status_t launch_gemm_bn(const CUtensorMap& ma, const CUtensorMap& mb, const 
   const int sms = num_sms();
   if (sms <= 0) return SQA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
-  kern<<<grid, sqa::kProjThreads, smem, st>>>(ma, mb, bias, c, M, K, N, accumulate);
-  return launch_status();
+  return launch_k(kern, dim3(grid), dim3(sqa::kProjThreads), smem, st, ma, mb, bias, c, M, K, N, accumulate);
 }
 
 template <bool kBf16, bool kAMN, bool kBMN>
@@ -594,23 +615,14 @@ sqa_status_t launch_decode(const void* q, const void* kc, const void* vc, const 
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
     return SQA_ERR_CUDA;
   dim3 grid(pl.n_split, static_cast<unsigned>(gy), B);
-  kern<<<grid, sqa::kDecThreads, C::kSmemBytes, st>>>(mq, mk, mv, p);
-  if (cudaGetLastError() != cudaSuccess) return SQA_ERR_CUDA;
+  const sqa_status_t s = launch_k(kern, grid, dim3(sqa::kDecThreads), C::kSmemBytes, st, mq, mk, mv, p);
+  if (s != SQA_OK) return s;
   if (pl.n_split > 1) {
     const size_t rows = static_cast<size_t>(B) * n_new * H_q;
-    // Launched as a programmatic dependent of the decode grid, so that its
-    // launch overlaps the decode grid's last CTAs.
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(rows));
-    cfg.blockDim = dim3(sqa::kCombineWarps * 32);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, sqa::decode_combine_kernel<D>, p) != cudaSuccess) return SQA_ERR_CUDA;
+    // Its launch overlaps the decode grid's last CTAs (which signal once
+    // their last load is issued).
+    return launch_k(sqa::decode_combine_kernel<D>, dim3(static_cast<unsigned>(rows)), dim3(sqa::kCombineWarps * 32),
+                    0, st, p);
   }
   return launch_status();
 }

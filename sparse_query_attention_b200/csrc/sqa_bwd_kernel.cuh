@@ -48,6 +48,8 @@ __global__ void bwd_prep_kernel(const void* __restrict__ o, int o_bf16, const __
                                 const float* __restrict__ lse, float* __restrict__ dsum, float* __restrict__ lse2,
                                 int B, int N, int H_q, int n_pad) {
   constexpr int kLanes = D / 8;  // 2 .. 16 lanes per row
+  grid_dependency_wait();  // O and LSE of the previous kernel on the stream are complete
+  grid_launch_dependents();
   const size_t gtid = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const size_t idx = gtid / kLanes;  // row of the padded [B, H_q, n_pad] space
   const int sub = static_cast<int>(gtid % kLanes);
@@ -264,9 +266,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tmem_alloc(&tmem_base_sh, 512);
     tmem_relinquish();
   }
+  // Programmatic dependent launch: the set-up above may overlap the end of
+  // the previous kernel on the stream; nothing below touches global memory
+  // before that kernel has completed.  Dependents are released only after
+  // the barrier, once this CTA holds its TMEM: a dependent CTA that took the
+  // SM's columns first would wait for this grid while this CTA waited for
+  // the columns.
+  grid_dependency_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  grid_launch_dependents();
   const uint32_t tmem = tmem_base_sh;
 
   if (warp < 4) {
@@ -657,9 +667,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tmem_alloc(&tmem_base_sh, 512);
     tmem_relinquish();
   }
+  // Programmatic dependent launch: the set-up above may overlap the end of
+  // the previous kernel on the stream; nothing below touches global memory
+  // before that kernel has completed.  Dependents are released only after
+  // the barrier, once this CTA holds its TMEM: a dependent CTA that took the
+  // SM's columns first would wait for this grid while this CTA waited for
+  // the columns.
+  grid_dependency_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  grid_launch_dependents();
   const uint32_t tmem = tmem_base_sh;
 
   if (warp < 4) {

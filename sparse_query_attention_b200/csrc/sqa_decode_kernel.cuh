@@ -93,6 +93,10 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   const int j = blockIdx.y / p.n_sub;
   const int sub = blockIdx.y % p.n_sub;
   const int b = blockIdx.z;
+  // Programmatic dependent launch: the previous kernel on the stream (which
+  // may have written the cache, the lengths or read this workspace) is
+  // complete before anything touches global memory.
+  grid_dependency_wait();
   const int len = decode_len(p, b, threadIdx.x == 0 && split == 0 && blockIdx.y == 0);
   const int kstart = split * p.chunk;
   if (kstart >= len) return;  // the whole CTA: this chunk lies past the sequence
@@ -398,6 +402,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32) decode_combine_kernel(cons
   const size_t n_rows = static_cast<size_t>(p.B) * p.n_new * p.H_q;
   const size_t row = blockIdx.x;  // grid = n_rows
   grid_dependency_wait();          // the partial results of the decode grid are complete
+  grid_launch_dependents();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int head = static_cast<int>(row % p.H_q);

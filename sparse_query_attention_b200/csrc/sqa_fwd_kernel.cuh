@@ -152,9 +152,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
+  // Programmatic dependent launch: the set-up above may overlap the end of
+  // the previous kernel on the stream; nothing below touches global memory
+  // before that kernel has completed.  Dependents are released only after
+  // the barrier, once this CTA holds its TMEM: a dependent CTA that took the
+  // SM's columns first would wait for this grid while this CTA waited for
+  // the columns.
+  grid_dependency_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  grid_launch_dependents();
   const uint32_t tmem = tmem_base_sh;
   // Registers: the block launches with 384 x 168; the producer/MMA
   // warpgroup needs few, the two softmax warpgroups hold a 128-column score
