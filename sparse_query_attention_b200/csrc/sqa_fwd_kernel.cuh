@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
       bool ok = mbar_wait(&q_full, 0, &abort_flag);
       // Step 0 scores.
-      int kslot = 0;  // ring position of K_i is 2i, of V_i is 2i + 1
+      // Ring positions: K_i at 2i, V_i at 2i + 1.
       if (ok) ok = mbar_wait(&slot_full[0], 0, &abort_flag);
       if (ok) {
         tc_fence_after();
@@ -278,7 +278,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           mma_commit_w(&slot_empty[ks]);
         }
       }
-      (void)kslot;
       mma_commit_w(&mma_done);
     }
   }
@@ -296,12 +295,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const float sl2 = p.scale_log2;
     const int tile_tok_min = t0 + t * T;
     const int tile_tok_max = min(tile_tok_min + T, p.N) - 1;
-    const int my_steps = n_steps;  // both tiles step in lock-step with the MMA warp
+    // Both tiles step in lock-step with the MMA warp, n_steps each.
 
     float m_used = -INFINITY;  // running max in log2 units (of scaled scores)
     float l_sum = 0.f;
     bool ok = true;
-    for (int i = 0; i < my_steps; ++i) {
+    for (int i = 0; i < n_steps; ++i) {
       if (!mbar_wait(&s_full[t], i & 1, &abort_flag)) {
         ok = false;
         break;
