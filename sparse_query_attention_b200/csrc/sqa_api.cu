@@ -15,6 +15,7 @@
 #include "sqa_decode_kernel.cuh"
 #include "sqa_fwd_kernel.cuh"
 #include "sqa_fwd_quad_kernel.cuh"
+#include "sqa_fwd_split_kernel.cuh"
 #include "sqa_proj_kernel.cuh"
 #include "sqa_ptx.cuh"
 
@@ -255,6 +256,28 @@ sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* ou
       return SQA_ERR_CUDA;
     return launch_k(kern, grid, dim3(sqa::kQuadThreads), sqa::QuadCfg<D>::kSmemBytes, st, mq, mk, mv, p);
   } else {
+    // Waves of the two-tile grid against the split grid (one query tile per
+    // CTA, its two tiles on the even and odd key blocks, half the work per
+    // CTA): the split kernel when its waves, halved, come out shorter.
+    // Unmasked problems only: under a band mask the work per CTA varies and
+    // the longest-first order already packs the waves (causal B=4, N=8192,
+    // (8,4) ran 2 % slower split).
+    const int sms = num_sms();
+    if (sms <= 0) return SQA_ERR_CUDA;
+    const int n_tblk1 = (N + T - 1) / T;
+    const long long ctas2 = static_cast<long long>(p.n_tblk) * gy * B;
+    const long long ctas1 = static_cast<long long>(n_tblk1) * gy * B;
+    const double waves2 = static_cast<double>((ctas2 + sms - 1) / sms);
+    const double waves1 = 0.5 * static_cast<double>((ctas1 + sms - 1) / sms);
+    if (!a.masked && waves1 < 0.97 * waves2) {
+      p.n_tblk = n_tblk1;
+      dim3 grid1(n_tblk1, static_cast<unsigned>(gy), B);
+      auto kern = sqa::sqa_fwd_split_kernel<D>;
+      constexpr int smem = sqa::SplitCfg<D>::kSmemBytes;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return SQA_ERR_CUDA;
+      return launch_k(kern, grid1, dim3(sqa::kFwdThreads), smem, st, mq, mk, mv, p);
+    }
     auto kern = sqa::sqa_fwd_kernel<D>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
       return SQA_ERR_CUDA;
