@@ -744,9 +744,11 @@ def run_profile(args):
 
     dev = torch.device("cuda", 0)
     stream = torch.cuda.current_stream(dev)
-    if args.profile == "fwd":
+    if args.profile in ("fwd", "xsqa"):
         w = WORKLOAD
         B, N, H_q, H_kv, d = w["B"], w["N"], w["H_q"], w["H_kv"], w["d_head"]
+        if args.profile == "xsqa":  # the encoder workload's xSQA variant (split kernel)
+            H_q, H_kv = VARIANTS["xSQA"]
         x = attention_inputs(B, N, H_q, H_kv, d, seed=2, device=dev)
         out = torch.empty((B, N, H_q * d), dtype=torch.float32, device=dev)
         for _ in range(args.steps):
@@ -783,8 +785,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["sqa", "reference"], default="sqa")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["fwd", "bwd", "decode"], default=None,
+    ap.add_argument("--profile", choices=["fwd", "xsqa", "bwd", "decode"], default=None,
                     help="only launch the kernels (for ncu): fwd = the bench workload's forward, "
+                         "xsqa = its xSQA (4,4) variant, "
                          "bwd = the B=4, N=8192 causal training step, decode = one SQA decode step of "
                          "B=16 sequences x 32768 cached tokens; no timing, no JSON")
     args = ap.parse_args(argv)
