@@ -867,6 +867,6 @@ const char* sqa_status_string(sqa_status_t status) {
   return "SQA_ERR_UNKNOWN";
 }
 
-const char* sqa_version(void) { return "0.2.0"; }
+const char* sqa_version(void) { return "0.3.0"; }
 
 }  // extern "C"
