@@ -21,7 +21,10 @@
  *    library allocates no device memory and keeps no per-call state.
  *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
  *    NULL means the legacy default stream).  Nothing synchronises except
- *    sqa_device_status().
+ *    sqa_device_status().  Kernels are launched as programmatic dependents
+ *    of the previous kernel on the stream: they may start their set-up
+ *    while it finishes but touch no global memory before it has completed,
+ *    so stream order holds for every buffer, as with ordinary launches.
  *  - Layouts are dense, row-major, with the last index contiguous:
  *      Q, O, dO, dQ : [B, N, H_q,  d_head]
  *      K, V, dK, dV : [B, N, H_kv, d_head]
