@@ -18,7 +18,12 @@
 // their running max and sum,
 //   m = max(m_a, m_b),  l = l_a 2^(m_a - m) + l_b 2^(m_b - m),
 //   O = (O_a 2^(m_a - m) + O_b 2^(m_b - m)) / l,  LSE = (m + log2 l) ln 2,
-// the same merge a split of the key range always admits.
+// the same merge a split of the key range always admits.  With four
+// softmax warpgroups the single MMA-issuing warp becomes the limit: every
+// tcgen05.mma costs ~55 cycles to issue whatever its size, and a step issues
+// 32 small ones (N = 64); merging or splitting that issue was measured
+// slower (one N = 128 score MMA per query tile couples the key halves; two
+// issuing warps contend).
 //
 // Roles (20 warps):
 //   warp 0 (one lane)  TMA: Q tiles once, then K_i, V_i into a ring of slots.
