@@ -385,6 +385,39 @@ DECODE = {"B": 16, "L": 32768, "n_new": 1, "d_head": 128}
 DECODE_VARIANTS = {"MHA": (16, 16), "GQA": (16, 4), "SQA": (8, 4), "xSQA": (4, 4), "xSMQA": (4, 1)}
 
 
+PROJ = {"M": 32768, "N": 4096, "K": 4096}
+
+
+def proj_operands(torch, dev):
+    g = torch.Generator(device=dev)
+    g.manual_seed(6)
+    c = PROJ
+    x = torch.randn((c["M"], c["K"]), generator=g, device=dev).to(torch.bfloat16)
+    w = (0.02 * torch.randn((c["N"], c["K"]), generator=g, device=dev)).to(torch.bfloat16)
+    return x, w
+
+
+def time_projection(sqa, torch, stream, dev, reps=10):
+    """The projection GEMM (Y = X W^T, bf16 in, bf16 out, fp32 accumulate) at
+    M=32768, N=K=4096, against torch.matmul (cuBLAS) on the same operands, as
+    context for the measured bf16 peak.  Operands (0.5 GB) exceed the L2."""
+    c = PROJ
+    M, N, K = c["M"], c["N"], c["K"]
+    x, w = proj_operands(torch, dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ours = lambda: sqa.sqa_proj(x, w, None, y, sqa.SQA_DT_BF16, M, K, N, stream=stream)
+    ref = lambda: torch.matmul(x, w.t(), out=y)
+    for _ in range(3):
+        ours()
+        ref()
+    t_ours, t_ref = device_times(torch, stream, [ours, ref], reps)
+    flops = 2.0 * M * N * K
+    ms_o, ms_r = statistics.median(t_ours), statistics.median(t_ref)
+    sqa.sqa_device_status(stream)
+    return {"config": dict(c), "sqa_proj_ms": ms_o, "sqa_proj_tflops": flops / ms_o / 1e9,
+            "cublas_ms": ms_r, "cublas_tflops": flops / ms_r / 1e9}
+
+
 def load_hbm_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -698,6 +731,7 @@ def run_sqa(args):
     windowed = time_windowed(sqa, torch, stream, dev)
     decode = time_decode(sqa, torch, stream, dev)
     cross = time_cross(sqa, torch, stream, dev)
+    projection = time_projection(sqa, torch, stream, dev)
 
     peak, peak_kind = load_peaks()
     achieved = flops_step / (statistics.mean(per_launch_ms) / 1e3) / 1e12
@@ -723,6 +757,7 @@ def run_sqa(args):
         "windowed": windowed,
         "decode": decode,
         "cross": cross,
+        "projection": projection,
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -754,6 +789,12 @@ def run_profile(args):
         for _ in range(args.steps):
             sqa.sqa_attn_fwd(x["q"], x["k"], x["v"], out, B, N, H_q, H_kv, d, w["causal"], 1 / math.sqrt(d),
                              stream=stream)
+    elif args.profile == "gemm":
+        c = PROJ
+        x, w = proj_operands(torch, dev)
+        y = torch.empty((c["M"], c["N"]), dtype=torch.bfloat16, device=dev)
+        for _ in range(args.steps):
+            sqa.sqa_proj(x, w, None, y, sqa.SQA_DT_BF16, c["M"], c["K"], c["N"], stream=stream)
     elif args.profile == "decode":
         c = DECODE
         B, L, n_new, d = c["B"], c["L"], c["n_new"], c["d_head"]
@@ -785,9 +826,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["sqa", "reference"], default="sqa")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["fwd", "xsqa", "bwd", "decode"], default=None,
+    ap.add_argument("--profile", choices=["fwd", "xsqa", "bwd", "decode", "gemm"], default=None,
                     help="only launch the kernels (for ncu): fwd = the bench workload's forward, "
-                         "xsqa = its xSQA (4,4) variant, "
+                         "xsqa = its xSQA (4,4) variant, gemm = the M=32768, N=K=4096 projection GEMM, "
                          "bwd = the B=4, N=8192 causal training step, decode = one SQA decode step of "
                          "B=16 sequences x 32768 cached tokens; no timing, no JSON")
     args = ap.parse_args(argv)
