@@ -78,8 +78,9 @@ def test_packed_bf16_gradients_fill_the_whole_buffer(sqa):
     rq, rk, rv = attention_backward(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(x["do"]), True, 0.125)
     # bf16 gradients: dV of the first keys sums P dO over up to N rows and 4
     # heads and reaches |dV| ~ 8-16, where one bf16 rounding alone is up to
-    # 2^-9 * 16 = 0.031; the bound is therefore taken relative to the
-    # tensor's scale (max|err| <= 2e-2 * max(1, max|ref|), relL2 <= 1e-2).
-    assert_close_scaled(f64(dqkv[:, :, :H_q]), rq, "dQ")
+    # 2^-9 * 16 = 0.031; for dK and dV the bound is therefore taken relative
+    # to the tensor's scale (max|err| <= 2e-2 * max(1, max|ref|), relL2 <=
+    # 1e-2).  dQ stays near unit size and takes the plain bound.
+    assert_close(f64(dqkv[:, :, :H_q]), rq, "dQ")
     assert_close_scaled(f64(dqkv[:, :, H_q:H_q + H_kv]), rk, "dK")
     assert_close_scaled(f64(dqkv[:, :, H_q + H_kv:]), rv, "dV")
