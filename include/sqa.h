@@ -252,7 +252,10 @@ sqa_status_t sqa_attn_bwd_packed(const void* qkv, const void* out, sqa_dtype_t o
  * Shapes whose workspace (sqa_attn_bwd_workspace_size) exceeds
  * SQA_BWD_STATIC_SCRATCH_BYTES return SQA_ERR_UNSUPPORTED and launch nothing.
  * The first call on a device looks up the array's device address (with that
- * device current); make that first call before any stream capture.  All
+ * device current); make that first call before any stream capture.  The
+ * address belongs to the device's context: after a cudaDeviceReset the next
+ * call finds a new context and looks the address up again (so, again, not
+ * inside a stream capture).  All
  * calls share the one array: calls that overlap on the GPU (different
  * streams, or different host threads, on the same device) race on it, so
  * serialise them.  The array keeps the previous call's contents; the

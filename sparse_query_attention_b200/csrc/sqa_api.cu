@@ -785,7 +785,9 @@ sqa_status_t sqa_attn_bwd_packed(const void* qkv, const void* out, sqa_dtype_t o
 // array, present on every GPU that loads the library until the process exits.
 // In host code `g_bwd_static_scratch` names a host-side shadow, never the
 // device memory: its device address comes from cudaGetSymbolAddress, looked
-// up once per device with that device current.
+// up with the device current, once per device and context.  A device reset
+// (cudaDeviceReset) destroys the context and with it the module's memory;
+// the next call sees a new context ID and looks the address up again.
 // ---------------------------------------------------------------------------
 static __device__ __align__(256) uint8_t g_bwd_static_scratch[SQA_BWD_STATIC_SCRATCH_BYTES];
 
@@ -793,16 +795,46 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_static_scratch_mu;
 void* g_static_scratch_addr[kMaxDevices] = {};
+unsigned long long g_static_scratch_ctx[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device, or null.
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_id = nullptr;
+std::once_flag g_ctx_fn_once;
+
+// Unique ID of the calling thread's current context, 0 if unknown.
+unsigned long long current_context_id() {
+  std::call_once(g_ctx_fn_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(fn);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (g_ctx_current == nullptr || g_ctx_id == nullptr || g_ctx_current(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+      g_ctx_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the scratch array in the current device's context, or
+// null.  Looked up again whenever the context differs from the one the
+// cached address belongs to (or when the context cannot be identified).
 void* static_scratch_on_current_device() {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lock(g_static_scratch_mu);
-  if (g_static_scratch_addr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (g_static_scratch_addr[dev] == nullptr || ctx == 0 || ctx != g_static_scratch_ctx[dev]) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_bwd_static_scratch) != cudaSuccess) return nullptr;
     g_static_scratch_addr[dev] = ptr;
+    g_static_scratch_ctx[dev] = current_context_id();  // the lookup makes the primary context current
   }
   return g_static_scratch_addr[dev];
 }
