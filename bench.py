@@ -90,7 +90,14 @@ def device_times(torch, stream, fns, reps, before=None):
     return [[ev[k].elapsed_time(ev[k + 1]) for ev in marks] for k in range(len(fns))]
 
 
+# Nominal dense bf16 tensor peak of a B200 (NVIDIA's sparse figure halved).
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
 def load_peaks():
+    """The roofline denominator: the measured cuBLAS bf16 burst rate of this
+    pool's B200s (MEASURED_PEAKS.json), else the earlier measurement on the
+    pool that stands in for it (1590 TFLOP/s)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as f:
@@ -128,27 +135,76 @@ def load_traffic():
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+    """SM clock and clock-event reasons sampled while the timed region runs:
+    an NVML query every 5 ms from a background thread (a short timed region
+    still gets tens of samples); nvidia-smi every 100 ms where NVML is not
+    available.  Only reads the GPU's state."""
 
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, period_s=0.005):
         self.gpu = gpu_index
+        self.period = period_s
+        self.samples = []  # (sm_mhz, reason bitmask)
+        self.sm_max = None
         self.proc = None
+        self.thread = None
+        self.source = None
+
+    def _nvml_loop(self, nv, handle):
+        import time as _t
+        while not self._stop:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                except AttributeError:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(handle)
+                self.samples.append((float(sm), int(rs)))
+            except Exception:  # noqa: BLE001
+                pass
+            _t.sleep(self.period)
 
     def __enter__(self):
+        self._stop = False
+        try:
+            import threading
+
+            import pynvml as nv
+            nv.nvmlInit()
+            handle = nv.nvmlDeviceGetHandleByIndex(self._physical_index())
+            self.sm_max = float(nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM))
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, handle), daemon=True)
+            self.thread.start()
+            self.source = "nvml every 5 ms"
+            return self
+        except Exception:  # noqa: BLE001
+            self.thread = None
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                ["nvidia-smi", "-i", str(self._physical_index()), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.source = "nvidia-smi every 100 ms"
         except OSError:
             self.proc = None
         return self
 
+    def _physical_index(self):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        parts = [p.strip() for p in vis.split(",") if p.strip()]
+        if parts and parts[0].isdigit() and self.gpu < len(parts):
+            return int(parts[self.gpu])
+        return self.gpu
+
     def __exit__(self, *exc):
-        self.lines = []
+        self._stop = True
+        if self.thread is not None:
+            self.thread.join(timeout=2)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -156,26 +212,31 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
                 out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            names = [n for n, _ in self.REASONS[:4]]
+            for ln in out.splitlines():
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm = float(parts[1])
+                    self.sm_max = float(parts[2])
+                except ValueError:
+                    continue
+                mask = 0
+                for (n, bit), val in zip(self.REASONS[:4], parts[5:9]):
+                    if val.lower() == "active":
+                        mask |= bit
+                self.samples.append((sm, mask))
+            del names
         return False
 
     def summary(self):
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-            except ValueError:
-                continue
-            for n, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        sm = [s for s, _ in self.samples]
+        reasons = sorted({n for _, m in self.samples for n, bit in self.REASONS if m & bit})
+        counts = {n: sum(1 for _, m in self.samples if m & bit) for n, bit in self.REASONS}
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.sm_max,
+                "reasons": reasons, "samples": len(sm), "source": self.source,
+                "reason_samples": {k: v for k, v in counts.items() if v}}
 
 
 # ----------------------------------------------------------------------------
@@ -205,6 +266,96 @@ def cpu_baseline(rows_per_head=6144, seed=2):
             "sample": f"{len(rows)} query rows x {w['H_q']} heads of the N={w['N']} workload "
                       f"({flops / 1e9:.1f} GFLOP, {dt:.2f} s, fp64 numpy)",
             "seconds": dt, "tokens_per_s": w["B"] * len(rows) / dt}
+
+
+def cpu_baseline_configs():
+    """The oracle timed on every configuration of the hot path, on this
+    host's cores, within about half a minute: the small causal core (B=2,
+    N=256, (4,2), d=32) in full; the decoder layer (B=16, N=1024,
+    d_model=256, d=16) forward in full for each of its five head-count
+    variants, its backward in full for SQA; the training step (B=4, N=8192,
+    (8,4), d=64, forward and backward) on one of its 16 independent
+    (batch, KV head) problems, extrapolated x16; the N=32768 encoder core on
+    64 sampled query rows per variant and the N=131072 / 200000 core (SQA,
+    xSQA) on 4 sampled rows, extrapolated linearly to all N rows (rows are
+    independent).  The oracle's inputs at N=131072 and 200000 for MHA's 16
+    heads would need several GB of fp64 K and V, so that variant is not
+    timed there.  Seconds are per configuration (per step for the layer)."""
+    import numpy as np
+    from oracle import attention_backward, attention_forward, sqa_layer_backward, sqa_layer_forward
+    from sqa_inputs import attention_inputs, layer_inputs, sample_rows
+
+    def np64(t):
+        return t.double().numpy()
+
+    out = {}
+    x = attention_inputs(2, 256, 4, 2, 32, 0, device="cpu")
+    q, k, v = (np64(x[n]) for n in ("q", "k", "v"))
+    t0 = time.perf_counter()
+    attention_forward(q, k, v, True, 1 / math.sqrt(32))
+    out["causal_core_b2_n256"] = {"timed": "full", "fwd_seconds": time.perf_counter() - t0}
+    c = LAYER
+    B, N, dm, dh = c["B"], c["N"], c["d_model"], c["d_head"]
+    lay = {}
+    for name in ("GQA", "SQA", "sSQA", "xSQA", "xSMQA"):
+        hq, hkv = LAYER_VARIANTS[name]
+        xl = layer_inputs(B, N, dm, hq, hkv, dh, seed=1, device="cpu")
+        a = [np64(xl[k]) for k in ("x", "wq", "wk", "wv", "wo")]
+        t0 = time.perf_counter()
+        sqa_layer_forward(*a, B, N, hq, hkv, dh, causal=True)
+        lay[name] = {"fwd_seconds": time.perf_counter() - t0}
+        if name == "SQA":
+            dy = np.random.default_rng(11).standard_normal((B * N, dm))
+            t0 = time.perf_counter()
+            sqa_layer_backward(*a, dy, B, N, hq, hkv, dh, causal=True)
+            lay[name]["bwd_seconds"] = time.perf_counter() - t0
+    out["decoder_layer_b16_n1024"] = {"timed": "full (backward for SQA only)", "variants": lay}
+    t = TRAIN
+    G = t["H_q"] // t["H_kv"]
+    xt = attention_inputs(1, t["N"], t["H_q"], t["H_kv"], t["d_head"], 4, with_dout=True, device="cpu")
+    q, do = (np64(xt[n][:, :, :G]) for n in ("q", "do"))  # KV head 0 and its G query heads
+    k, v = (np64(xt[n][:, :, :1]) for n in ("k", "v"))
+    sc = 1 / math.sqrt(t["d_head"])
+    parts = t["B"] * t["H_kv"]
+    t0 = time.perf_counter()
+    attention_forward(q, k, v, True, sc)
+    t1 = time.perf_counter()
+    attention_backward(q, k, v, do, True, sc)
+    t2 = time.perf_counter()
+    out["training_step_b4_n8192"] = {"timed": f"1 of {parts} (batch, KV head) problems, extrapolated x{parts}",
+                                     "fwd_seconds": parts * (t1 - t0), "bwd_seconds": parts * (t2 - t1)}
+    del xt, q, k, v, do
+    w = WORKLOAD
+    enc = {}
+    rows = sample_rows(w["N"], 64, 2)
+    for name, (hq, hkv) in VARIANTS.items():
+        xe = attention_inputs(1, w["N"], hq, hkv, w["d_head"], 2, device="cpu")
+        q, k, v = (np64(xe[n]) for n in ("q", "k", "v"))
+        del xe
+        t0 = time.perf_counter()
+        attention_forward(q, k, v, False, 1 / math.sqrt(w["d_head"]), rows=rows)
+        dt = time.perf_counter() - t0
+        enc[name] = {"fwd_seconds": dt * w["N"] / len(rows), "sample_seconds": dt}
+        del q, k, v
+    out["encoder_core_n32768"] = {"timed": f"{len(rows)} sampled query rows, extrapolated to N={w['N']}",
+                                  "variants": enc}
+    lng = {}
+    for N in LONG["N"]:
+        rows = sample_rows(N, 4, 3)
+        per = {}
+        for name in ("SQA", "xSQA"):
+            hq, hkv = LONG_VARIANTS[name]
+            xe = attention_inputs(1, N, hq, hkv, LONG["d_head"], 3, device="cpu")
+            q, k, v = (np64(xe[n]) for n in ("q", "k", "v"))
+            del xe
+            t0 = time.perf_counter()
+            attention_forward(q, k, v, False, 1 / math.sqrt(LONG["d_head"]), rows=rows)
+            dt = time.perf_counter() - t0
+            per[name] = {"fwd_seconds": dt * N / len(rows), "sample_seconds": dt}
+            del q, k, v
+        lng[str(N)] = per
+    out["long_core"] = {"timed": "4 sampled query rows, extrapolated to N (MHA not timed)", "by_N": lng}
+    return out
 
 
 def run_reference(args):
@@ -252,19 +403,27 @@ def time_long_sequences(sqa, torch, stream, dev, reps=3):
     d = c["d_head"]
     res = {}
     for N in c["N"]:
-        per = {}
+        # The variants are timed round-robin (one launch each per round) so
+        # that the speed-up over MHA compares launches at the same clock.
+        data, fns = {}, []
         for name, (hq, hkv) in LONG_VARIANTS.items():
             x = attention_inputs(1, N, hq, hkv, d, seed=3, device=dev)
             o = torch.empty((1, N, hq * d), dtype=torch.float32, device=dev)
-            def fwd():
+            data[name] = (x, o)
+
+            def fwd(x=x, o=o, hq=hq, hkv=hkv):
                 sqa.sqa_attn_fwd(x["q"], x["k"], x["v"], o, 1, N, hq, hkv, d, False, 1 / math.sqrt(d),
                                  stream=stream)
 
             fwd()
-            ms = statistics.median(device_times(torch, stream, [fwd], reps)[0])
+            fns.append(fwd)
+        times = device_times(torch, stream, fns, reps)
+        per = {}
+        for (name, (hq, hkv)), t in zip(LONG_VARIANTS.items(), times):
+            ms = statistics.median(t)
             per[name] = {"H_q": hq, "H_kv": hkv, "ms": ms,
                          "tflops": attn_fwd_flops(1, N, hq, d, False) / ms / 1e9, "tokens_per_s": N / (ms / 1e3)}
-            del x, o
+        del data, fns
         for name in per:
             per[name]["speedup_vs_mha"] = per["MHA"]["ms"] / per[name]["ms"]
         res[str(N)] = per
@@ -646,7 +805,7 @@ def run_sqa(args):
     ho = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
     dsets = [tuple(torch.empty_like(t) for t in (x["q"], x["k"], x["v"])) for _ in range(2)]
     douts = [torch.empty_like(out) for _ in range(2)]
-    e2e_steps = max(3, min(args.steps, 10))
+    e2e_steps = max(10, min(args.steps, 50))
 
     def serial_step():
         dq_, dk_, dv_ = dsets[0]
@@ -709,18 +868,34 @@ def run_sqa(args):
     d2h = ho[0].numel() * ho[0].element_size()
 
     # --- head-count variants on the same kernel (speed-up vs H_q = H) ------
-    variants = {}
+    # Timed round-robin, one launch of every variant per round (L2 flushed
+    # before each): on a GPU at its power cap the clock drifts over tens of
+    # milliseconds, and variants timed one block after another would compare
+    # different clocks.
+    vin = {}
     for name, (vq, vkv) in VARIANTS.items():
         xv = attention_inputs(B, N, vq, vkv, d, seed=2, device=dev)
-        ov = torch.empty((B, N, vq * d), dtype=torch.float32, device=dev)
+        vin[name] = (xv, torch.empty((B, N, vq * d), dtype=torch.float32, device=dev))
         for _ in range(2):
-            step(xv["q"], xv["k"], xv["v"], ov, vq, vkv)
-        times = device_times(torch, stream, [lambda: step(xv["q"], xv["k"], xv["v"], ov, vq, vkv)], 5,
-                             before=lambda: flush.fill_(1))[0]
-        ms = statistics.median(times)
-        variants[name] = {"H_q": vq, "H_kv": vkv, "ms": ms,
-                          "tflops": attn_fwd_flops(B, N, vq, d, w["causal"]) / (ms / 1e3) / 1e12}
-        del xv, ov
+            step(xv["q"], xv["k"], xv["v"], vin[name][1], vq, vkv)
+    names = list(VARIANTS)
+
+    def launcher(nm):
+        vq, vkv = VARIANTS[nm]
+        xv, ov = vin[nm]
+        return lambda: step(xv["q"], xv["k"], xv["v"], ov, vq, vkv)
+
+    fns = []
+    for nm in names:  # a flush, then the launch: one timed interval per variant per round
+        fns += [lambda: flush.fill_(1), launcher(nm)]
+    rounds = device_times(torch, stream, fns, 7)
+    variants = {}
+    for i, nm in enumerate(names):
+        vq, vkv = VARIANTS[nm]
+        ms = statistics.median(rounds[2 * i + 1])
+        variants[nm] = {"H_q": vq, "H_kv": vkv, "ms": ms,
+                        "tflops": attn_fwd_flops(B, N, vq, d, w["causal"]) / (ms / 1e3) / 1e12}
+    del vin
     for name in variants:
         variants[name]["speedup_vs_mha"] = variants["MHA"]["ms"] / variants[name]["ms"]
         variants[name]["ideal_speedup"] = VARIANTS["MHA"][0] / variants[name]["H_q"]
@@ -744,6 +919,7 @@ def run_sqa(args):
                        l2="flushed between timed steps (256 MiB write)"),
         "tokens_per_s": tokens_per_s,
         "pct_of_bf16_peak": 100 * achieved / peak,
+        "pct_of_nominal_bf16_peak": 100 * achieved / NOMINAL_BF16_TFLOPS,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_source": f"{peak_kind} bf16 burst"},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -762,6 +938,7 @@ def run_sqa(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = {k: v for k, v in cpu_baseline().items() if k not in ("seconds",)}
+        line["cpu_baseline"]["configs"] = cpu_baseline_configs()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -779,11 +956,11 @@ def run_profile(args):
 
     dev = torch.device("cuda", 0)
     stream = torch.cuda.current_stream(dev)
-    if args.profile in ("fwd", "xsqa"):
+    if args.profile in ("fwd", "xsqa", "mha", "gqa"):
         w = WORKLOAD
         B, N, H_q, H_kv, d = w["B"], w["N"], w["H_q"], w["H_kv"], w["d_head"]
-        if args.profile == "xsqa":  # the encoder workload's xSQA variant (split kernel)
-            H_q, H_kv = VARIANTS["xSQA"]
+        if args.profile != "fwd":  # another head-count variant of the encoder workload
+            H_q, H_kv = VARIANTS[{"xsqa": "xSQA", "mha": "MHA", "gqa": "GQA"}[args.profile]]
         x = attention_inputs(B, N, H_q, H_kv, d, seed=2, device=dev)
         out = torch.empty((B, N, H_q * d), dtype=torch.float32, device=dev)
         for _ in range(args.steps):
@@ -826,9 +1003,10 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["sqa", "reference"], default="sqa")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["fwd", "xsqa", "bwd", "decode", "gemm"], default=None,
+    ap.add_argument("--profile", choices=["fwd", "xsqa", "mha", "gqa", "bwd", "decode", "gemm"], default=None,
                     help="only launch the kernels (for ncu): fwd = the bench workload's forward, "
-                         "xsqa = its xSQA (4,4) variant, gemm = the M=32768, N=K=4096 projection GEMM, "
+                         "xsqa / mha / gqa = its xSQA (4,4), MHA (16,16) or GQA (16,4) variant, "
+                         "gemm = the M=32768, N=K=4096 projection GEMM, "
                          "bwd = the B=4, N=8192 causal training step, decode = one SQA decode step of "
                          "B=16 sequences x 32768 cached tokens; no timing, no JSON")
     args = ap.parse_args(argv)
