@@ -516,24 +516,35 @@ def time_cross(sqa, torch, stream, dev, reps=5):
         fn()
         return statistics.median(device_times(torch, stream, [fn], reps)[0])
 
-    res = {}
+    # Forward of the three variants timed round-robin (one launch of each
+    # per round), then the SQA backward.
+    res, data, fns = {}, {}, []
+    BF = sqa.SQA_DT_BF16
     for name, (hq, hkv) in LONG_VARIANTS.items():
         x = cross_attention_inputs(B, Nq, Nkv, hq, hkv, d, seed=6, with_dout=name == "SQA", device=dev)
         o = torch.empty((B, Nq, hq, d), dtype=torch.bfloat16, device=dev)
         lse = torch.empty((B, hq, Nq), dtype=torch.float32, device=dev)
-        BF = sqa.SQA_DT_BF16
-        ms = med(lambda: sqa.sqa_attn_fwd_cross(x["q"], x["k"], x["v"], o, BF, lse, B, Nq, Nkv, hq, hkv, d, sc,
-                                                stream=stream))
+        data[name] = (x, o, lse)
+
+        def fwd(x=x, o=o, lse=lse, hq=hq, hkv=hkv):
+            sqa.sqa_attn_fwd_cross(x["q"], x["k"], x["v"], o, BF, lse, B, Nq, Nkv, hq, hkv, d, sc, stream=stream)
+
+        fwd()
+        fns.append(fwd)
+    times = device_times(torch, stream, fns, reps)
+    for (name, (hq, hkv)), t in zip(LONG_VARIANTS.items(), times):
+        ms = statistics.median(t)
         flops = 4 * B * hq * Nq * Nkv * d
         res[name] = {"H_q": hq, "H_kv": hkv, "fwd_ms": ms, "fwd_tflops": flops / ms / 1e9}
-        if name == "SQA":
-            dq, dk, dv = (torch.empty(t.shape, dtype=torch.bfloat16, device=dev) for t in (x["q"], x["k"], x["v"]))
-            wsb = sqa.sqa_attn_bwd_workspace_size(B, Nq, hq, hkv, d)
-            ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
-            bms = med(lambda: sqa.sqa_attn_bwd_cross(x["q"], x["k"], x["v"], o, BF, x["do"], lse, dq, dk, dv, BF, B,
-                                                     Nq, Nkv, hq, hkv, d, sc, ws, wsb, stream=stream))
-            res[name].update({"bwd_ms": bms, "bwd_tflops": 2 * flops / bms / 1e9})
-        del x, o, lse
+    x, o, lse = data["SQA"]
+    hq, hkv = LONG_VARIANTS["SQA"]
+    dq, dk, dv = (torch.empty(t.shape, dtype=torch.bfloat16, device=dev) for t in (x["q"], x["k"], x["v"]))
+    wsb = sqa.sqa_attn_bwd_workspace_size(B, Nq, hq, hkv, d)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    bms = med(lambda: sqa.sqa_attn_bwd_cross(x["q"], x["k"], x["v"], o, BF, x["do"], lse, dq, dk, dv, BF, B, Nq, Nkv,
+                                             hq, hkv, d, sc, ws, wsb, stream=stream))
+    res["SQA"].update({"bwd_ms": bms, "bwd_tflops": 8 * B * hq * Nq * Nkv * d / bms / 1e9})
+    del data, fns
     for name in res:
         res[name]["fwd_speedup_vs_mha"] = res["MHA"]["fwd_ms"] / res[name]["fwd_ms"]
     sqa.sqa_device_status(stream)

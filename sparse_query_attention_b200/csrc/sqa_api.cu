@@ -243,6 +243,8 @@ sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* ou
   p.win_l = a.win_l;
   p.win_r = a.win_r;
   p.longest_first = a.longest_first;
+  p.tblk0 = 0;
+  p.wait_at_exit = 0;
   p.out_bf16 = out_bf16;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const long long gy = static_cast<long long>(H_kv) * p.n_sub;
@@ -256,27 +258,52 @@ sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* ou
       return SQA_ERR_CUDA;
     return launch_k(kern, grid, dim3(sqa::kQuadThreads), sqa::QuadCfg<D>::kSmemBytes, st, mq, mk, mv, p);
   } else {
-    // Waves of the two-tile grid against the split grid (one query tile per
-    // CTA, its two tiles on the even and odd key blocks, half the work per
-    // CTA): the split kernel when its waves, halved, come out shorter.
-    // Unmasked problems only: under a band mask the work per CTA varies and
-    // the longest-first order already packs the waves (causal B=4, N=8192,
-    // (8,4) ran 2 % slower split).
+    // Three ways to cover an unmasked problem's query tiles, chosen by their
+    // wave counts on this GPU's SMs (one CTA per SM): the two-tile grid (two
+    // query tiles per CTA); the split grid (one tile per CTA, its two
+    // softmax tiles on the even and odd key blocks, so half the work per CTA
+    // at a rate measured ~8 % lower: a split wave costs kSplitWave of a
+    // two-tile wave); or both, the two-tile kernel on the token blocks that
+    // fill whole waves and the split kernel on the remaining tiles, launched
+    // after it on the stream (its CTAs start on the SMs the last two-tile
+    // wave frees, and wait for that grid only before exiting).  Under a band mask the work per CTA varies and the
+    // longest-first order already packs the waves (causal B=4, N=8192, (8,4)
+    // ran 2 % slower split), so masked problems keep the two-tile grid.
     const int sms = num_sms();
     if (sms <= 0) return SQA_ERR_CUDA;
-    const int n_tblk1 = (N + T - 1) / T;
-    const long long ctas2 = static_cast<long long>(p.n_tblk) * gy * B;
-    const long long ctas1 = static_cast<long long>(n_tblk1) * gy * B;
-    const double waves2 = static_cast<double>((ctas2 + sms - 1) / sms);
-    const double waves1 = 0.5 * static_cast<double>((ctas1 + sms - 1) / sms);
-    if (!a.masked && waves1 < 0.97 * waves2) {
-      p.n_tblk = n_tblk1;
-      dim3 grid1(n_tblk1, static_cast<unsigned>(gy), B);
+    constexpr double kSplitWave = 0.55;
+    const long long yz = gy * B;
+    const int n_tiles = (N + T - 1) / T;
+    auto waves = [&](long long ctas) { return static_cast<double>((ctas + sms - 1) / sms); };
+    const double t_two = waves(static_cast<long long>(p.n_tblk) * yz);
+    const double t_split = kSplitWave * waves(static_cast<long long>(n_tiles) * yz);
+    // mixed: the largest number of token blocks whose two-tile CTAs fill whole waves
+    const int n_a = static_cast<int>((static_cast<long long>(p.n_tblk) * yz / sms) * sms / yz);
+    const double t_mix = n_a > 0 && n_a < p.n_tblk
+                             ? waves(static_cast<long long>(n_a) * yz) +
+                                   kSplitWave * waves(static_cast<long long>(n_tiles - 2 * n_a) * yz)
+                             : 1e30;
+    auto launch_split = [&](int tile0, int tiles) -> sqa_status_t {
+      sqa::FwdParams ps = p;
+      ps.n_tblk = n_tiles;
+      ps.tblk0 = tile0;
+      ps.wait_at_exit = tile0 > 0;  // after the two-tile launch of the same problem
+      dim3 grid1(tiles, static_cast<unsigned>(gy), B);
       auto kern = sqa::sqa_fwd_split_kernel<D>;
       constexpr int smem = sqa::SplitCfg<D>::kSmemBytes;
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return SQA_ERR_CUDA;
-      return launch_k(kern, grid1, dim3(sqa::kFwdThreads), smem, st, mq, mk, mv, p);
+      return launch_k(kern, grid1, dim3(sqa::kFwdThreads), smem, st, mq, mk, mv, ps);
+    };
+    if (!a.masked && t_split < 0.97 * t_two && t_split <= t_mix) return launch_split(0, n_tiles);
+    if (!a.masked && t_mix < 0.97 * t_two) {
+      auto kern = sqa::sqa_fwd_kernel<D>;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+        return SQA_ERR_CUDA;
+      dim3 grid_a(n_a, static_cast<unsigned>(gy), B);
+      const sqa_status_t s2 = launch_k(kern, grid_a, dim3(sqa::kFwdThreads), C::kSmemBytes, st, mq, mk, mv, p);
+      if (s2 != SQA_OK) return s2;
+      return launch_split(2 * n_a, n_tiles - 2 * n_a);
     }
     auto kern = sqa::sqa_fwd_kernel<D>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)

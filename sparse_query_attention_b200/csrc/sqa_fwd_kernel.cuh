@@ -65,6 +65,8 @@ struct FwdParams {
   int masked;      // band mask active (causal or sliding window)
   int win_l, win_r;  // band: t - win_l <= u <= t + win_r (both <= N)
   int longest_first;  // schedule token blocks from the last one
+  int tblk0;          // first token block of this launch (a problem may be split over two launches)
+  int wait_at_exit;   // second launch of a split problem: wait for the previous grid only before exiting
   int out_bf16;
   float scale_log2;  // scale * log2(e)
 };
@@ -103,7 +105,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   // ---- work unit -----------------------------------------------------------
   const int T = 128 >> p.log2g;  // tokens per tile
   const BlockUnit u = block_unit(p.longest_first);
-  const int tblk = p.longest_first ? (p.n_tblk - 1 - u.x) : u.x;
+  const int tblk = p.tblk0 + (p.longest_first ? (p.n_tblk - 1 - u.x) : u.x);
   const int j = u.y / p.n_sub;
   const int sub = u.y % p.n_sub;
   const int b = u.z;

@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   // ---- work unit -----------------------------------------------------------
   const int T = 128 >> p.log2g;  // tokens per tile
   const BlockUnit u = block_unit(p.longest_first);
-  const int tblk = p.longest_first ? (p.n_tblk - 1 - u.x) : u.x;
+  const int tblk = p.tblk0 + (p.longest_first ? (p.n_tblk - 1 - u.x) : u.x);
   const int j = u.y / p.n_sub;
   const int sub = u.y % p.n_sub;
   const int b = u.z;
@@ -120,7 +120,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   // the barrier, once this CTA holds its TMEM: a dependent CTA that took the
   // SM's columns first would wait for this grid while this CTA waited for
   // the columns.
-  grid_dependency_wait();
+  // Exception (wait_at_exit): launched right after the two-tile kernel on the
+  // other query tiles of the same problem, this grid reads only Q, K and V,
+  // which the two-tile grid had already waited for before it released this
+  // one, and writes rows that grid does not touch; so its CTAs start work at
+  // once on the SMs that grid's last wave frees, and wait for that grid only
+  // before they exit, so that this grid completes after it and the next
+  // launch's wait covers both.
+  if (!p.wait_at_exit) grid_dependency_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -454,6 +461,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
+  if (p.wait_at_exit) grid_dependency_wait();
 }
 
 }  // namespace sqa

@@ -160,6 +160,26 @@ def test_long_sequence_sampled_rows_per_head(sqa, N, H_q, H_kv):
         assert_close(f64(lse[0, h, ri]), lse_ref[0, 0], f"LSE head {h}")
 
 
+@pytest.mark.parametrize("N,H_q,H_kv,boundary", [(40883, 4, 4, 148 * 2 * 128), (32768, 4, 1, 444 * 2 * 32)])
+def test_mixed_grid_boundary_rows(sqa, N, H_q, H_kv, boundary):
+    """Unmasked d = 128 problems whose two-tile grid leaves a mostly empty
+    last wave run the two-tile kernel on the token blocks that fill whole
+    waves and the split kernel on the rest (148 SMs: 40883 tokens of xSQA,
+    boundary at token 37888; 32768 tokens of (4,1), four heads packed per
+    tile, boundary at token 28416).  Rows on both sides of the boundary, in
+    the ragged last tile and sampled elsewhere, against the oracle."""
+    d = 128
+    x = attention_inputs(1, N, H_q, H_kv, d, seed=41, device="cuda")
+    o, lse = run_fwd(sqa, x["q"], x["k"], x["v"], False)
+    sqa.sqa_device_status()
+    edge = [0, 1, boundary - 2, boundary - 1, boundary, boundary + 1, N - 2, N - 1]
+    rows = np.unique(np.concatenate([sample_rows(N, 96, seed=41), np.array(edge)]))
+    ri = torch.as_tensor(rows, device="cuda")
+    o_ref, lse_ref = _oracle_fwd(x, False, rows=rows)
+    assert_close(f64(o[:, ri]), o_ref, "O rows")
+    assert_close(f64(lse[:, :, ri]), lse_ref, "LSE rows")
+
+
 def test_fwd_deterministic(sqa):
     x = attention_inputs(1, 1000, 8, 4, 64, seed=12, device="cuda")
     o1, l1 = run_fwd(sqa, x["q"], x["k"], x["v"], True)

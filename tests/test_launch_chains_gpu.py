@@ -33,12 +33,16 @@ def _fwd(sqa, x, out, causal):
                         1 / math.sqrt(d))
 
 
-@pytest.mark.parametrize("d,causal", [(64, True), (128, False), (16, True)])
-def test_forward_then_projection_chain(sqa, d, causal):
+@pytest.mark.parametrize("d,causal,B,N,H_q,H_kv", [(64, True, 2, 640, 8, 4), (128, False, 2, 640, 8, 4),
+                                                   (16, True, 2, 640, 8, 4), (128, False, 1, 40883, 4, 4)])
+def test_forward_then_projection_chain(sqa, d, causal, B, N, H_q, H_kv):
     """fwd(X_s) -> O, then Y_s = O W^T, for three inputs through ONE O
     buffer: each projection reads the O just written, and the next forward
-    overwrites O right after that projection was launched."""
-    B, N, H_q, H_kv, Nout = 2, 640, 8, 4, 96
+    overwrites O right after that projection was launched.  The last shape
+    runs the forward as two launches (two-tile kernel, then the split kernel
+    on the remaining query tiles, which waits for the first only before it
+    exits)."""
+    Nout = 96
     xs = [attention_inputs(B, N, H_q, H_kv, d, seed=900 + s, device="cuda") for s in range(3)]
     g = torch.Generator(device="cuda")
     g.manual_seed(901)
