@@ -500,6 +500,40 @@ sqa_status_t launch_gemm_bn(const CUtensorMap& ma, const CUtensorMap& mb, const 
   return launch_k(kern, dim3(grid), dim3(sqa::kProjThreads), smem, st, ma, mb, bias, c, M, K, N, accumulate);
 }
 
+// CTA-pair GEMM (K-contiguous A and B): clusters of two, persistent over the
+// 256 x 256 output tiles, as many pairs as can be resident at once.
+template <bool kBf16>
+sqa_status_t launch_gemm_pair(const CUtensorMap& ma, const CUtensorMap& mb, const float* bias, void* c, int M, int N,
+                              int K, int accumulate, cudaStream_t st) {
+  auto kern = sqa::proj_gemm_pair_kernel<kBf16>;
+  constexpr int smem = sqa::kPairDynamicBytes;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return SQA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.blockDim = dim3(sqa::kProjThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int max_pairs = 0;
+  cfg.gridDim = dim3(2 * 64);
+  if (cudaOccupancyMaxActiveClusters(&max_pairs, kern, &cfg) != cudaSuccess || max_pairs <= 0) return SQA_ERR_CUDA;
+  const long long tiles = static_cast<long long>((M + 2 * kProjBM - 1) / (2 * kProjBM)) *
+                          ((N + sqa::kPairBN - 1) / sqa::kPairBN);
+  const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, ma, mb, bias, c, M, K, N, accumulate) == cudaSuccess ? SQA_OK
+                                                                                              : SQA_ERR_CUDA;
+}
+
 template <bool kBf16, bool kAMN, bool kBMN>
 sqa_status_t launch_gemm_layouts(const CUtensorMap& ma, const CUtensorMap& mb, int bn, const float* bias, void* c,
                                  int M, int N, int K, int accumulate, cudaStream_t st) {
@@ -541,6 +575,19 @@ sqa_status_t gemm_impl(const void* a, bool a_mn, const void* b, bool b_mn, const
     return SQA_ERR_CUDA;
   cudaStream_t st = as_stream(stream);
   const bool bf = c_dtype == SQA_DT_BF16;
+  // Large K-contiguous products (the layer's forward projections, nn.Linear
+  // layout) run on CTA pairs with 256 x 256 tiles when there are enough tiles
+  // to occupy every pair of SMs.
+  const int sms = num_sms();
+  const long long pair_tiles = static_cast<long long>((M + 2 * kProjBM - 1) / (2 * kProjBM)) *
+                               ((N + sqa::kPairBN - 1) / sqa::kPairBN);
+  if (!a_mn && !b_mn && N >= sqa::kPairBN && sms > 0 && pair_tiles >= sms / 2) {
+    CUtensorMap mb2;
+    const uint32_t b2_box[2] = {64, uint32_t(kProjBM)};  // each CTA loads 128 of the tile's 256 B rows
+    if (!make_map_bf16(&mb2, b, 2, b_dims, b_strides, b2_box)) return SQA_ERR_CUDA;
+    return bf ? launch_gemm_pair<true>(ma, mb2, bias, c, M, N, K, accumulate, st)
+              : launch_gemm_pair<false>(ma, mb2, bias, c, M, N, K, accumulate, st);
+  }
   if (!a_mn && !b_mn)
     return bf ? launch_gemm_layouts<true, false, false>(ma, mb, bn, bias, c, M, N, K, accumulate, st)
               : launch_gemm_layouts<false, false, false>(ma, mb, bn, bias, c, M, N, K, accumulate, st);

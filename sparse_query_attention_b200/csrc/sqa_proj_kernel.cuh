@@ -265,4 +265,216 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   }
 }
 
+// ===========================================================================
+// The same GEMM over CTA pairs, for K-contiguous A and B (activations times
+// nn.Linear weights, the layer's forward projections): 256 x 256 output
+// tiles, one per pair.  Each CTA loads its own 128 rows of A and 128 of the
+// 256 rows of B (output columns) per 64-wide K slice, 32 KB instead of the
+// 48 KB a single CTA needs for a 128 x 256 tile, so six stages fit and the
+// ring covers ~1.5x the L2 latency of the single-CTA kernel.  The even CTA's
+// MMA warp issues one tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16) per
+// K step; both CTAs' copies complete on the even CTA's "full" barrier, the
+// even CTA's commits arrive on both CTAs' "empty" and accumulator barriers,
+// and both CTAs' epilogue warps arrive on the even CTA's accumulator-free
+// barrier.  Each CTA's epilogue writes its own 128 rows from its own TMEM.
+// ===========================================================================
+constexpr int kPairBN = 256;  // output columns per pair tile (128 per CTA's B half)
+constexpr int kPairStages = 6;
+constexpr int kPairHalfBytes = kProjBM * kProjBK * 2;  // 16 KB: A rows or B rows of one CTA, one K slice
+constexpr int kPairDynamicBytes = kPairStages * 2 * kPairHalfBytes + 1024;
+
+template <bool kOutBf16>
+__global__ void __launch_bounds__(kProjThreads, 1)
+    proj_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                          const float* __restrict__ bias, void* __restrict__ y, int M, int K, int Nout,
+                          int accumulate) {
+  constexpr uint32_t kAccCols = kPairBN;       // one accumulator: 128 lanes x 256 columns per CTA
+  constexpr uint32_t kTmemCols = 2 * kAccCols;  // two, alternating per tile
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[kPairStages];   // used in the even CTA
+  __shared__ __align__(8) uint64_t empty_bar[kPairStages];  // both
+  __shared__ __align__(8) uint64_t acc_full[2];             // both
+  __shared__ __align__(8) uint64_t acc_empty[2];            // used in the even CTA
+  __shared__ __align__(8) uint64_t mma_done;                // both
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* a_tiles = smem;
+  uint8_t* b_tiles = smem + kPairStages * kPairHalfBytes;
+
+  const int warp = warp_id_uniform();
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int pair = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+  const int m_tiles = (M + 2 * kProjBM - 1) / (2 * kProjBM);
+  const int n_tiles = (Nout + kPairBN - 1) / kPairBN;
+  const int num_tiles = m_tiles * n_tiles;
+  const int num_kb = (K + kProjBK - 1) / kProjBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 8);  // four epilogue warps in each CTA
+    }
+    mbar_init(&mma_done, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc_pair(&tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  if (warp == 1 && lane == 0) {
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+  }
+  // Programmatic dependent launch as in proj_gemm_kernel; the cluster
+  // barrier makes both CTAs' barrier initialisation and TMEM allocation
+  // visible to the pair before either uses the other's.
+  grid_dependency_wait();
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  grid_launch_dependents();
+  const uint32_t tmem = tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // TMA producer of this CTA; g counts k-blocks over the pair's tiles.
+      const uint32_t full0 = map_to_rank(&full_bar[0], 0);  // the even CTA's full barriers
+      int g = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += n_pairs) {
+        int mt, nt;
+        proj_tile_coords(tile, m_tiles, n_tiles, mt, nt);
+        const int m0 = mt * 2 * kProjBM + static_cast<int>(rank) * kProjBM;
+        const int n0 = nt * kPairBN + static_cast<int>(rank) * kProjBM;
+        for (int kb = 0; kb < num_kb; ++kb, ++g) {
+          const int s = g % kPairStages;
+          const uint32_t ph = (g / kPairStages) & 1;
+          if (g >= kPairStages && !mbar_wait(&empty_bar[s], ph ^ 1, &abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 4 * kPairHalfBytes);  // both CTAs' A and B
+          const uint32_t fb = full0 + s * static_cast<uint32_t>(sizeof(uint64_t));
+          tma_load_2d_pair(&tm_a, fb, a_tiles + s * kPairHalfBytes, kb * kProjBK, m0);
+          tma_load_2d_pair(&tm_b, fb, b_tiles + s * kPairHalfBytes, kb * kProjBK, n0);
+        }
+      }
+      // No copy of this CTA may still be landing in its shared memory when
+      // it exits: the even CTA drains its full barriers (which count both
+      // CTAs' copies); the odd CTA's last copies are covered by the MMAs
+      // that consumed them (mma_done) or, after an abort, by the final
+      // cluster barrier following the even CTA's drain.
+      if (rank == 0)
+        for (int q = g > kPairStages ? g - kPairStages : 0; q < g; ++q)
+          mbar_drain(&full_bar[q % kPairStages], (q / kPairStages) & 1);
+    }
+  } else if (warp == 1) {
+    if (rank == 0) {
+      // MMA issuer of the pair: the whole warp runs the loop, one lane issues.
+      constexpr uint32_t idesc = idesc_bf16_f32(2 * kProjBM, kPairBN, 0, 0);
+      const uint64_t a_desc0 = smem_desc(smem_addr(a_tiles), 16, 1024, kSw128);
+      const uint64_t b_desc0 = smem_desc(smem_addr(b_tiles), 16, 1024, kSw128);
+      int g = 0;
+      bool ok = true;
+      for (int tile = pair, k = 0; tile < num_tiles && ok; tile += n_pairs, ++k) {
+        const int acc = k & 1;
+        // Both CTAs' epilogues have read this accumulator's previous tile.
+        if (k >= 2 && !mbar_wait(&acc_empty[acc], ((k >> 1) - 1) & 1, &abort_flag)) break;
+        tc_fence_after();
+        const uint32_t tacc = tmem + acc * kAccCols;
+        for (int kb = 0; kb < num_kb; ++kb, ++g) {
+          const int s = g % kPairStages;
+          const uint32_t ph = (g / kPairStages) & 1;
+          if (!mbar_wait(&full_bar[s], ph, &abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = desc_advance(a_desc0, s * kPairHalfBytes);
+          const uint64_t bd = desc_advance(b_desc0, s * kPairHalfBytes);
+#pragma unroll
+          for (int kk = 0; kk < kProjBK / 16; ++kk)
+            mma_ss_pair_w(tacc, desc_advance(ad, kk * 32), desc_advance(bd, kk * 32), idesc, (kb | kk) != 0);
+          mma_commit_pair_w(&empty_bar[s]);
+        }
+        if (ok) mma_commit_pair_w(&acc_full[acc]);
+      }
+      mma_commit_pair_w(&mma_done);
+    }
+  } else if (warp >= 4) {
+    // Epilogue: warp w reads TMEM lanes [32 (w - 4), +32) = this CTA's output rows.
+    const int wq = warp & 3;
+    const uint32_t acc_empty0 = map_to_rank(&acc_empty[0], 0);
+    for (int tile = pair, k = 0; tile < num_tiles; tile += n_pairs, ++k) {
+      const int acc = k & 1;
+      if (!mbar_wait(&acc_full[acc], (k >> 1) & 1, &abort_flag)) break;
+      tc_fence_after();
+      int mt, nt;
+      proj_tile_coords(tile, m_tiles, n_tiles, mt, nt);
+      const int row = mt * 2 * kProjBM + static_cast<int>(rank) * kProjBM + wq * 32 + lane;
+      const int n0 = nt * kPairBN;
+      const uint32_t lane_addr = tmem + acc * kAccCols + (static_cast<uint32_t>(wq * 32) << 16);
+#pragma unroll 1
+      for (int c0 = 0; c0 < kPairBN; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(lane_addr + c0, r);
+        tmem_wait_ld();
+        const int n = n0 + c0;
+        if (row < M && n < Nout) {
+          float v[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]) + (bias != nullptr ? bias[n + i] : 0.f);
+          if constexpr (kOutBf16) {
+            uint4* dst =
+                reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(y) + static_cast<size_t>(row) * Nout + n);
+            dst[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                                pack_bf16x2(v[6], v[7]));
+            dst[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
+                                pack_bf16x2(v[14], v[15]));
+          } else {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(y) + static_cast<size_t>(row) * Nout + n);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              float4 w = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+              if (accumulate) {
+                const float4 old = dst[i];
+                w.x += old.x;
+                w.y += old.y;
+                w.z += old.z;
+                w.w += old.w;
+              }
+              dst[i] = w;
+            }
+          }
+        }
+      }
+      // Hand the accumulator back to the even CTA's MMA warp.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(acc_empty0 + acc * static_cast<uint32_t>(sizeof(uint64_t)));
+    }
+  }
+
+  // ---- teardown: every MMA of the pair has finished, in both CTAs ----------
+  __syncwarp();
+  if (threadIdx.x == 32) mbar_drain(&mma_done, 0);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA leaves while the other may still arrive on its barriers
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
 }  // namespace sqa

@@ -119,7 +119,7 @@ __device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
 }
 
 // ---------------------------------------------------------------------------
-// TMA (cp.async.bulk.tensor), no multicast.
+// TMA (cp.async.bulk.tensor): each load writes this CTA's shared memory only.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -323,6 +323,80 @@ __device__ __forceinline__ void tmem_st_words(uint32_t taddr, const uint32_t (&r
   if constexpr (N == 8) tmem_st8(taddr, r);
   if constexpr (N == 16) tmem_st16(taddr, r);
   if constexpr (N == 32) tmem_st32(taddr, r);
+}
+
+// ---------------------------------------------------------------------------
+// CTA pairs (cluster of two, cta_group::2).  One tcgen05.mma issued by the
+// even CTA of the pair computes an M = 256 tile: each CTA supplies 128 rows of
+// A from its own shared memory (or TMEM) and half of the N columns of B, and
+// holds its 128 rows of the accumulator in its own TMEM.  Every tcgen05
+// instruction of a kernel that uses pairs takes the cta_group::2 form.  Each
+// TMA load below writes one CTA's own shared memory only.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Arrive-release / wait-acquire on the cluster barrier: every thread of both
+// CTAs of the pair must reach it.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// The shared::cluster address of the same shared-memory location in CTA
+// `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+  return r;
+}
+// Arrive on an mbarrier in another CTA of the cluster (shared::cluster address).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// 2-D TMA load into this CTA's shared memory whose completion is counted on
+// an mbarrier of either CTA of the pair (shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* map, uint32_t bar_cluster, void* dst, int c0,
+                                                 int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+      "[%2];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem] over the pair (M = 256): issued by the even
+// CTA; whole warp, one elected lane.
+__device__ __forceinline__ void mma_ss_pair_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, l;\n\t"
+      "elect.sync _|l, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@l tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on the mbarrier at this shared-memory offset in both CTAs of
+// the pair when every MMA issued so far by this thread has completed.
+__device__ __forceinline__ void mma_commit_pair_w(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred l;\n\t"
+      "elect.sync _|l, 0xffffffff;\n\t"
+      "@l tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n\t}\n" ::
+          "r"(smem_addr(bar)),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
 }
 
 // ---------------------------------------------------------------------------

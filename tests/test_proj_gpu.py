@@ -57,6 +57,54 @@ def test_proj_bias_and_bf16(sqa):
     assert_close(f64(y), projection(f64(x), f64(w), f64(bias)), "Y")
 
 
+@pytest.mark.parametrize("M,K,Nout,bf16_out", [(4100, 528, 2320, True), (4100, 528, 2320, False),
+                                                (2048, 4096, 512, True)])
+def test_proj_pair_tiles(sqa, M, K, Nout, bf16_out):
+    """Products large enough to run on CTA pairs (256 x 256 tiles, two SMs per
+    tile): ragged M, Nout and K (M not a multiple of 256, Nout of 256, K of
+    64), with a bias."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed(M + 3 * K + Nout)
+    x = torch.randn((M, K), generator=g, device="cuda").to(torch.bfloat16)
+    w = (torch.randn((Nout, K), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    bias = torch.randn((Nout,), generator=g, device="cuda")
+    y = _proj(sqa, x, w, bias=bias, out_dtype=torch.bfloat16 if bf16_out else torch.float32)
+    sqa.sqa_device_status()
+    assert_close(f64(y), projection(f64(x), f64(w), f64(bias)), "Y")
+
+
+def test_gemm_pair_tiles_accumulate(sqa):
+    """C += A B^T twice into an fp32 C on the pair path (sqa_gemm, both
+    operands K-contiguous): the epilogue adds to what C holds."""
+    M, K, N = 3000, 256, 1024
+    g = torch.Generator(device="cuda")
+    g.manual_seed(77)
+    a = torch.randn((M, K), generator=g, device="cuda").to(torch.bfloat16)
+    b = (torch.randn((N, K), generator=g, device="cuda") * 0.05).to(torch.bfloat16)
+    c0 = torch.randn((M, N), generator=g, device="cuda")
+    c = c0.clone()
+    KC = sqa.SQA_K_CONTIGUOUS
+    sqa.sqa_gemm(a, KC, b, KC, None, c, sqa.SQA_DT_F32, True, M, N, K)
+    sqa.sqa_gemm(a, KC, b, KC, None, c, sqa.SQA_DT_F32, True, M, N, K)
+    sqa.sqa_device_status()
+    assert_close(f64(c), f64(c0) + 2 * projection(f64(a), f64(b)), "C")
+
+
+def test_proj_bench_size_sampled_rows(sqa):
+    """The bench's projection, M = 32768, N = K = 4096, bf16 out, on the pair
+    path; 256 seeded rows against the oracle."""
+    M, K, N = 32768, 4096, 4096
+    g = torch.Generator(device="cuda")
+    g.manual_seed(6)
+    x = torch.randn((M, K), generator=g, device="cuda").to(torch.bfloat16)
+    w = (0.02 * torch.randn((N, K), generator=g, device="cuda")).to(torch.bfloat16)
+    y = _proj(sqa, x, w, out_dtype=torch.bfloat16)
+    sqa.sqa_device_status()
+    rows = np.sort(np.random.default_rng(6).choice(M, 256, replace=False))
+    ri = torch.as_tensor(rows, device="cuda")
+    assert_close(f64(y[ri]), projection(f64(x[ri]), f64(w)), "Y rows")
+
+
 VARIANTS = {"GQA": (16, 4), "SQA": (8, 4), "sSQA": (8, 8), "xSQA": (4, 4), "xSMQA": (4, 1)}
 
 
