@@ -485,6 +485,19 @@ sqa_status_t attn_bwd_impl(const void* q, const void* k, const void* v, const vo
 // ---------------------------------------------------------------------------
 // Projection GEMM
 // ---------------------------------------------------------------------------
+// Raster of the persistent GEMMs (row tiles per group of the tile walk):
+// the smaller operand stays resident in L2 while the other streams through
+// once.  kResident leaves most of the 126 MB L2 (two halves, one per die) to
+// the streamed operand's tiles in flight and to the output.
+int gemm_group_m(int M, int N, int K, int bm) {
+  constexpr long long kResident = 40ll << 20;
+  const long long a_bytes = 2ll * M * K;
+  const long long b_bytes = 2ll * N * K;
+  if (b_bytes <= kResident && b_bytes <= a_bytes) return 1;  // N fastest: B stays
+  if (a_bytes <= kResident) return (M + bm - 1) / bm;        // M fastest: A stays
+  return 8;  // both large: groups of 8 row tiles share each pass over B
+}
+
 template <int BN, bool kBf16, bool kAMN, bool kBMN>
 sqa_status_t launch_gemm_bn(const CUtensorMap& ma, const CUtensorMap& mb, const float* bias, void* c, int M, int N,
                             int K, int accumulate, cudaStream_t st) {
@@ -497,7 +510,8 @@ sqa_status_t launch_gemm_bn(const CUtensorMap& ma, const CUtensorMap& mb, const 
   const int sms = num_sms();
   if (sms <= 0) return SQA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
-  return launch_k(kern, dim3(grid), dim3(sqa::kProjThreads), smem, st, ma, mb, bias, c, M, K, N, accumulate);
+  return launch_k(kern, dim3(grid), dim3(sqa::kProjThreads), smem, st, ma, mb, bias, c, M, K, N, accumulate,
+                  gemm_group_m(M, N, K, kProjBM));
 }
 
 // CTA-pair GEMM (K-contiguous A and B): clusters of two, persistent over the
@@ -530,8 +544,10 @@ sqa_status_t launch_gemm_pair(const CUtensorMap& ma, const CUtensorMap& mb, cons
   const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
   cfg.gridDim = dim3(2 * pairs);
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, ma, mb, bias, c, M, K, N, accumulate) == cudaSuccess ? SQA_OK
-                                                                                              : SQA_ERR_CUDA;
+  const int group_m = gemm_group_m(M, N, K, 2 * kProjBM);
+  return cudaLaunchKernelEx(&cfg, kern, ma, mb, bias, c, M, K, N, accumulate, group_m) == cudaSuccess
+             ? SQA_OK
+             : SQA_ERR_CUDA;
 }
 
 template <bool kBf16, bool kAMN, bool kBMN>

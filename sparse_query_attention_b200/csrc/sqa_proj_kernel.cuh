@@ -11,9 +11,9 @@
 // operand layout, so no transpose ever goes through memory.
 //
 // Design: a persistent kernel, one CTA per SM walking the 128 x BN output
-// tiles in groups of kProjGroupM row tiles (N fastest inside a group, so the
-// CTAs running together reuse a few A row tiles and the B tiles from L2
-// instead of streaming A once per column tile), eight warps:
+// tiles in groups of row tiles (all column tiles of a group before the next;
+// the group size is chosen so that the CTAs running together find their A
+// and B tiles in L2 and each operand comes from DRAM about once), eight warps:
 //   warp 0 / one lane : TMA producer, 64-wide K slices of A and B into a
 //                       4-stage ring (128-byte swizzle) that runs on across
 //                       tiles.
@@ -47,15 +47,18 @@ struct ProjSmem {
 // K-contiguous (A[m][k] / B[n][k]).  An MN-contiguous tile is loaded as
 // 64 (MN) x 64 (K) boxes, one 8 KB chunk per 64 rows of M or N.
 constexpr int kProjThreads = 256;
-constexpr int kProjGroupM = 8;  // row tiles per raster group
 
-// Output tile of linear index `tile`: groups of kProjGroupM row tiles, all
+// Output tile of linear index `tile`: groups of `group_m` row tiles, all
 // column tiles of a group before the next group, rows fastest inside it.
-__device__ __forceinline__ void proj_tile_coords(int tile, int m_tiles, int n_tiles, int& mt, int& nt) {
-  const int per_group = kProjGroupM * n_tiles;
+// group_m = 1 walks N fastest (every B tile stays hot in L2 while A streams
+// through once); group_m >= m_tiles walks M fastest (A stays, B streams once).
+// The host picks the raster from the operand sizes.
+__device__ __forceinline__ void proj_tile_coords(int tile, int m_tiles, int n_tiles, int group_m, int& mt,
+                                                 int& nt) {
+  const int per_group = group_m * n_tiles;
   const int group = tile / per_group;
-  const int first = group * kProjGroupM;
-  const int gm = min(kProjGroupM, m_tiles - first);
+  const int first = group * group_m;
+  const int gm = min(group_m, m_tiles - first);
   const int local = tile - group * per_group;
   mt = first + local % gm;
   nt = local / gm;
@@ -64,7 +67,8 @@ __device__ __forceinline__ void proj_tile_coords(int tile, int m_tiles, int n_ti
 template <int BN, bool kOutBf16, bool kAMN, bool kBMN>
 __global__ void __launch_bounds__(kProjThreads, 1)
     proj_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                     const float* __restrict__ bias, void* __restrict__ y, int M, int K, int Nout, int accumulate) {
+                     const float* __restrict__ bias, void* __restrict__ y, int M, int K, int Nout, int accumulate,
+                     int group_m) {
   static_assert(!kBMN || BN % 64 == 0, "MN-contiguous B needs BN in 64, 128, 256");
   using S = ProjSmem<BN>;
   constexpr uint32_t kAccCols = BN < 32 ? 32 : BN;  // one accumulator
@@ -131,7 +135,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         int mt, nt;
-        proj_tile_coords(tile, m_tiles, n_tiles, mt, nt);
+        proj_tile_coords(tile, m_tiles, n_tiles, group_m, mt, nt);
         const int m0 = mt * kProjBM;
         const int n0 = nt * BN;
         for (int kb = 0; kb < num_kb; ++kb, ++g) {
@@ -209,7 +213,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       if (!mbar_wait(&acc_full[acc], (k >> 1) & 1, &abort_flag)) break;
       tc_fence_after();
       int mt, nt;
-      proj_tile_coords(tile, m_tiles, n_tiles, mt, nt);
+      proj_tile_coords(tile, m_tiles, n_tiles, group_m, mt, nt);
       const int row = mt * kProjBM + wq * 32 + lane;
       const int n0 = nt * BN;
       const uint32_t lane_addr = tmem + acc * kAccCols + (static_cast<uint32_t>(wq * 32) << 16);
@@ -287,7 +291,7 @@ template <bool kOutBf16>
 __global__ void __launch_bounds__(kProjThreads, 1)
     proj_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                           const float* __restrict__ bias, void* __restrict__ y, int M, int K, int Nout,
-                          int accumulate) {
+                          int accumulate, int group_m) {
   constexpr uint32_t kAccCols = kPairBN;       // one accumulator: 128 lanes x 256 columns per CTA
   constexpr uint32_t kTmemCols = 2 * kAccCols;  // two, alternating per tile
   extern __shared__ uint8_t smem_raw[];
@@ -353,7 +357,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       bool ok = true;
       for (int tile = pair; tile < num_tiles && ok; tile += n_pairs) {
         int mt, nt;
-        proj_tile_coords(tile, m_tiles, n_tiles, mt, nt);
+        proj_tile_coords(tile, m_tiles, n_tiles, group_m, mt, nt);
         const int m0 = mt * 2 * kProjBM + static_cast<int>(rank) * kProjBM;
         const int n0 = nt * kPairBN + static_cast<int>(rank) * kProjBM;
         for (int kb = 0; kb < num_kb; ++kb, ++g) {
@@ -420,7 +424,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       if (!mbar_wait(&acc_full[acc], (k >> 1) & 1, &abort_flag)) break;
       tc_fence_after();
       int mt, nt;
-      proj_tile_coords(tile, m_tiles, n_tiles, mt, nt);
+      proj_tile_coords(tile, m_tiles, n_tiles, group_m, mt, nt);
       const int row = mt * 2 * kProjBM + static_cast<int>(rank) * kProjBM + wq * 32 + lane;
       const int n0 = nt * kPairBN;
       const uint32_t lane_addr = tmem + acc * kAccCols + (static_cast<uint32_t>(wq * 32) << 16);
