@@ -90,6 +90,8 @@ bool supported_d(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 
 // Streaming multiprocessors of the current device (looked up per call; the
 // attribute query is cheap and the current device may change).
+constexpr int kMaxDevices = 64;  // device ordinals with per-device host caches
+
 int num_sms() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -550,6 +552,103 @@ sqa_status_t launch_gemm_pair(const CUtensorMap& ma, const CUtensorMap& mb, cons
              : SQA_ERR_CUDA;
 }
 
+// Split K over clusters (proj_gemm_splitk_kernel): for products with few
+// output tiles and a long K.  Clusters of 8, 4 or 2 CTAs, the largest for
+// which one cluster per output tile fits on the device at once and each CTA
+// keeps at least four K blocks; 0 when none does.  How many clusters of a
+// size fit is queried once per device and size.
+template <int BN, bool kBf16, bool kAMN, bool kBMN>
+int gemm_split_count(long long tiles, int num_kb) {
+  static int max_clusters[kMaxDevices][3] = {};  // 0: not queried yet; -1: query failed
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  auto kern = sqa::proj_gemm_splitk_kernel<BN, kBf16, kAMN, kBMN>;
+  constexpr int smem = sqa::SplitSmem<BN>::kDynamicBytes;
+  for (int splits = 8, slot = 2; splits >= 2; splits /= 2, --slot) {
+    if (num_kb < 4 * splits) continue;
+    if (max_clusters[dev][slot] == 0) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 0;
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = splits;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(splits * 64);
+      cfg.blockDim = dim3(sqa::kProjThreads);
+      cfg.dynamicSmemBytes = smem;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      max_clusters[dev][slot] = cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0 ? n : -1;
+    }
+    if (tiles <= max_clusters[dev][slot]) return splits;
+  }
+  return 0;
+}
+
+template <int BN, bool kBf16, bool kAMN, bool kBMN>
+sqa_status_t launch_gemm_splitk(const CUtensorMap& ma, const CUtensorMap& mb, const float* bias, void* c, int M,
+                                int N, int K, int accumulate, int splits, cudaStream_t st) {
+  auto kern = sqa::proj_gemm_splitk_kernel<BN, kBf16, kAMN, kBMN>;
+  constexpr int smem = sqa::SplitSmem<BN>::kDynamicBytes;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return SQA_ERR_CUDA;
+  const long long tiles = static_cast<long long>((M + kProjBM - 1) / kProjBM) * ((N + BN - 1) / BN);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles * splits));
+  cfg.blockDim = dim3(sqa::kProjThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, ma, mb, bias, c, M, K, N, accumulate) == cudaSuccess ? SQA_OK
+                                                                                              : SQA_ERR_CUDA;
+}
+
+// Split-K dispatch for one layout pair: BN = 64, or 32 for a K-contiguous B
+// of at most 32 columns.  Sets *taken when it launched (or failed to).
+template <bool kAMN, bool kBMN>
+sqa_status_t gemm_splitk_layout(const void* a, const void* b, const uint64_t* a_dims, const uint64_t* a_strides,
+                                const uint32_t* a_box, const uint64_t* b_dims, const uint64_t* b_strides,
+                                const float* bias, void* c, bool bf, int M, int N, int K, int accumulate,
+                                cudaStream_t st, bool* taken) {
+  *taken = false;
+  const int bn = (!kBMN && N <= 32) ? 32 : 64;
+  const long long tiles = static_cast<long long>((M + kProjBM - 1) / kProjBM) * ((N + bn - 1) / bn);
+  const int num_kb = (K + sqa::kProjBK - 1) / sqa::kProjBK;
+  int splits = 0;
+  if (bn == 32) {
+    if constexpr (!kBMN)
+      splits = bf ? gemm_split_count<32, true, kAMN, kBMN>(tiles, num_kb)
+                  : gemm_split_count<32, false, kAMN, kBMN>(tiles, num_kb);
+  } else {
+    splits = bf ? gemm_split_count<64, true, kAMN, kBMN>(tiles, num_kb)
+                : gemm_split_count<64, false, kAMN, kBMN>(tiles, num_kb);
+  }
+  if (splits < 2) return SQA_OK;
+  *taken = true;
+  CUtensorMap ma, mb;
+  const uint32_t b_box[2] = {64, kBMN ? 64u : uint32_t(bn)};
+  if (!make_map_bf16(&ma, a, 2, a_dims, a_strides, a_box) || !make_map_bf16(&mb, b, 2, b_dims, b_strides, b_box))
+    return SQA_ERR_CUDA;
+  if (bn == 32) {
+    if constexpr (!kBMN)
+      return bf ? launch_gemm_splitk<32, true, kAMN, kBMN>(ma, mb, bias, c, M, N, K, accumulate, splits, st)
+                : launch_gemm_splitk<32, false, kAMN, kBMN>(ma, mb, bias, c, M, N, K, accumulate, splits, st);
+    return SQA_ERR_UNSUPPORTED;
+  }
+  return bf ? launch_gemm_splitk<64, true, kAMN, kBMN>(ma, mb, bias, c, M, N, K, accumulate, splits, st)
+            : launch_gemm_splitk<64, false, kAMN, kBMN>(ma, mb, bias, c, M, N, K, accumulate, splits, st);
+}
+
 template <bool kBf16, bool kAMN, bool kBMN>
 sqa_status_t launch_gemm_layouts(const CUtensorMap& ma, const CUtensorMap& mb, int bn, const float* bias, void* c,
                                  int M, int N, int K, int accumulate, cudaStream_t st) {
@@ -587,14 +686,34 @@ sqa_status_t gemm_impl(const void* a, bool a_mn, const void* b, bool b_mn, const
   const uint64_t b_dims[2] = {uint64_t(b_mn ? N : K), uint64_t(b_mn ? K : N)};
   const uint64_t b_strides[1] = {uint64_t(b_mn ? N : K) * 2};
   const uint32_t b_box[2] = {64, b_mn ? 64u : uint32_t(bn)};
-  if (!make_map_bf16(&ma, a, 2, a_dims, a_strides, a_box) || !make_map_bf16(&mb, b, 2, b_dims, b_strides, b_box))
-    return SQA_ERR_CUDA;
   cudaStream_t st = as_stream(stream);
   const bool bf = c_dtype == SQA_DT_BF16;
+  const int sms = num_sms();
+  // Few output tiles and a long K (a layer's weight gradients, K = tokens):
+  // split K over clusters instead of leaving most SMs idle.
+  const long long tiles = static_cast<long long>((M + kProjBM - 1) / kProjBM) * ((N + bn - 1) / bn);
+  if (sms > 0 && tiles * 4 <= sms && (K + sqa::kProjBK - 1) / sqa::kProjBK >= 8) {
+    bool taken = false;
+    sqa_status_t r = SQA_OK;
+    if (!a_mn && !b_mn)
+      r = gemm_splitk_layout<false, false>(a, b, a_dims, a_strides, a_box, b_dims, b_strides, bias, c, bf, M, N, K,
+                                           accumulate, st, &taken);
+    else if (!a_mn && b_mn)
+      r = gemm_splitk_layout<false, true>(a, b, a_dims, a_strides, a_box, b_dims, b_strides, bias, c, bf, M, N, K,
+                                          accumulate, st, &taken);
+    else if (a_mn && b_mn)
+      r = gemm_splitk_layout<true, true>(a, b, a_dims, a_strides, a_box, b_dims, b_strides, bias, c, bf, M, N, K,
+                                         accumulate, st, &taken);
+    else
+      r = gemm_splitk_layout<true, false>(a, b, a_dims, a_strides, a_box, b_dims, b_strides, bias, c, bf, M, N, K,
+                                          accumulate, st, &taken);
+    if (taken) return r;
+  }
+  if (!make_map_bf16(&ma, a, 2, a_dims, a_strides, a_box) || !make_map_bf16(&mb, b, 2, b_dims, b_strides, b_box))
+    return SQA_ERR_CUDA;
   // Large K-contiguous products (the layer's forward projections, nn.Linear
   // layout) run on CTA pairs with 256 x 256 tiles when there are enough tiles
   // to occupy every pair of SMs.
-  const int sms = num_sms();
   const long long pair_tiles = static_cast<long long>((M + 2 * kProjBM - 1) / (2 * kProjBM)) *
                                ((N + sqa::kPairBN - 1) / sqa::kPairBN);
   if (!a_mn && !b_mn && N >= sqa::kPairBN && sms > 0 && pair_tiles >= sms / 2) {
@@ -882,7 +1001,6 @@ sqa_status_t sqa_attn_bwd_packed(const void* qkv, const void* out, sqa_dtype_t o
 static __device__ __align__(256) uint8_t g_bwd_static_scratch[SQA_BWD_STATIC_SCRATCH_BYTES];
 
 namespace {
-constexpr int kMaxDevices = 64;
 std::mutex g_static_scratch_mu;
 void* g_static_scratch_addr[kMaxDevices] = {};
 unsigned long long g_static_scratch_ctx[kMaxDevices] = {};

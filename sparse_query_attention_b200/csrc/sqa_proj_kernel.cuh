@@ -481,4 +481,229 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   }
 }
 
+// ===========================================================================
+// Split K over a thread-block cluster, for products with few output tiles and
+// a long K: the weight gradients of a layer, dW = dY^T X, contract over all
+// B * N tokens into a d_model-sized tile grid that would otherwise leave all
+// but a few SMs idle.  Each cluster of S CTAs (S in 2, 4, 8) computes one
+// 128 x BN output tile; CTA r of the cluster contracts K blocks
+// [r num_kb / S, (r + 1) num_kb / S) into its TMEM accumulator.  Once its
+// last MMA has finished, each CTA stages its fp32 partial tile in its own
+// shared memory (over the operand ring, idle by then), and after a cluster
+// barrier CTA r sums rows [r 128 / S, (r + 1) 128 / S) of all S partials
+// through distributed shared memory, in rank order, and writes them (bias,
+// accumulate and output type as in proj_gemm_kernel).  The sum order is
+// fixed, so results are the same from run to run; no workspace is needed.
+// Warp roles as in proj_gemm_kernel, one tile per cluster; the ring is as
+// deep as ~192 KB of shared memory allows (up to 8 stages), since each CTA's
+// share of K is short and latency, not the tensor pipe, bounds it.
+// ===========================================================================
+template <int BN>
+struct SplitSmem {
+  static constexpr int kABytes = kProjBM * kProjBK * 2;
+  static constexpr int kBBytes = BN * kProjBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (192 * 1024 / kStageBytes) < 8 ? (192 * 1024 / kStageBytes) : 8;
+  static constexpr int kPartStride = BN + 4;  // floats per staged row; the pad spreads rows over the banks
+  static_assert(kProjBM * kPartStride * 4 <= kStages * kStageBytes, "the partial tile fits over the ring");
+  static constexpr int kDynamicBytes = kStages * kStageBytes + 1024;
+};
+
+template <int BN, bool kOutBf16, bool kAMN, bool kBMN>
+__global__ void __launch_bounds__(kProjThreads, 1)
+    proj_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                            const float* __restrict__ bias, void* __restrict__ y, int M, int K, int Nout,
+                            int accumulate) {
+  static_assert(BN % 16 == 0 && BN >= 32 && BN <= 64, "split-K tiles are 128 x 32 or 128 x 64");
+  static_assert(!kBMN || BN == 64, "MN-contiguous B is loaded as 64-column boxes");
+  using S = SplitSmem<BN>;
+  constexpr int kStages = S::kStages;
+  constexpr uint32_t kTmemCols = BN;  // one accumulator
+  constexpr uint32_t kMnChunk = 64 * 128;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[kStages];
+  __shared__ __align__(8) uint64_t empty_bar[kStages];
+  __shared__ __align__(8) uint64_t acc_full;
+  __shared__ __align__(8) uint64_t mma_done;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* a_tiles = smem;
+  uint8_t* b_tiles = smem + kStages * S::kABytes;
+  float* part = reinterpret_cast<float*>(smem);  // [128][kPartStride], once the ring is idle
+
+  const int warp = warp_id_uniform();
+  const int lane = threadIdx.x & 31;
+  const int splits = static_cast<int>(cluster_num_ctas());
+  const int rank = static_cast<int>(cluster_rank());
+  const int n_tiles = (Nout + BN - 1) / BN;
+  const int tile = static_cast<int>(blockIdx.x) / splits;
+  const int m0 = (tile / n_tiles) * kProjBM;
+  const int n0 = (tile % n_tiles) * BN;
+  const int num_kb = (K + kProjBK - 1) / kProjBK;
+  const int kb0 = static_cast<int>(static_cast<long long>(num_kb) * rank / splits);
+  const int kb1 = static_cast<int>(static_cast<long long>(num_kb) * (rank + 1) / splits);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&acc_full, 1);
+    mbar_init(&mma_done, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(&tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 1 && lane == 0) {
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+  }
+  // Programmatic dependent launch as in proj_gemm_kernel.
+  grid_dependency_wait();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  grid_launch_dependents();
+  const uint32_t tmem = tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // TMA producer over this CTA's K blocks.
+      int g = 0;
+      for (int kb = kb0; kb < kb1; ++kb, ++g) {
+        const int s = g % kStages;
+        if (g >= kStages && !mbar_wait(&empty_bar[s], ((g / kStages) & 1) ^ 1, &abort_flag)) break;
+        mbar_arrive_expect_tx(&full_bar[s], S::kABytes + S::kBBytes);
+        uint8_t* a_dst = a_tiles + s * S::kABytes;
+        uint8_t* b_dst = b_tiles + s * S::kBBytes;
+        if constexpr (kAMN) {
+          for (int c = 0; c < kProjBM / 64; ++c)
+            tma_load_2d(&tm_a, &full_bar[s], a_dst + c * kMnChunk, m0 + 64 * c, kb * kProjBK);
+        } else {
+          tma_load_2d(&tm_a, &full_bar[s], a_dst, kb * kProjBK, m0);
+        }
+        if constexpr (kBMN) {
+          tma_load_2d(&tm_b, &full_bar[s], b_dst, n0, kb * kProjBK);
+        } else {
+          tma_load_2d(&tm_b, &full_bar[s], b_dst, kb * kProjBK, n0);
+        }
+      }
+      // No copy may still be landing in shared memory once the ring is reused.
+      for (int q = g > kStages ? g - kStages : 0; q < g; ++q) mbar_drain(&full_bar[q % kStages], (q / kStages) & 1);
+    }
+  } else if (warp == 1) {
+    // MMA issuer (whole warp in the loop, lane 0 issues), as in proj_gemm_kernel.
+    constexpr uint32_t idesc = idesc_bf16_f32(kProjBM, BN, kAMN ? 1 : 0, kBMN ? 1 : 0);
+    const uint64_t a_desc0 = kAMN ? smem_desc(smem_addr(a_tiles), kMnChunk, 1024, kSw128)
+                                  : smem_desc(smem_addr(a_tiles), 16, 1024, kSw128);
+    const uint64_t b_desc0 = kBMN ? smem_desc(smem_addr(b_tiles), kMnChunk, 1024, kSw128)
+                                  : smem_desc(smem_addr(b_tiles), 16, 1024, kSw128);
+    constexpr uint32_t kAStep = kAMN ? 16 * 128 : 32;
+    constexpr uint32_t kBStep = kBMN ? 16 * 128 : 32;
+    bool ok = true;
+    int g = 0;
+    for (int kb = kb0; kb < kb1; ++kb, ++g) {
+      const int s = g % kStages;
+      if (!mbar_wait(&full_bar[s], (g / kStages) & 1, &abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint64_t ad = desc_advance(a_desc0, s * S::kABytes);
+      const uint64_t bd = desc_advance(b_desc0, s * S::kBBytes);
+#pragma unroll
+      for (int kk = 0; kk < kProjBK / 16; ++kk)
+        mma_ss_w(tmem, desc_advance(ad, kk * kAStep), desc_advance(bd, kk * kBStep), idesc, (g | kk) != 0);
+      mma_commit_w(&empty_bar[s]);
+    }
+    if (ok) mma_commit_w(&acc_full);
+    mma_commit_w(&mma_done);
+  } else if (warp >= 4) {
+    // Stage this CTA's partial tile: TMEM lane (row) -> its padded smem row.
+    // acc_full fires after the last MMA has finished reading the ring, and
+    // every copy into the ring was waited for before its MMA was issued.
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    if (mbar_wait(&acc_full, 0, &abort_flag)) {
+      tc_fence_after();
+      float* dst = part + row * S::kPartStride;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(lane_addr + c0, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          reinterpret_cast<float4*>(dst + c0)[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                                               __uint_as_float(r[4 * i + 2]),
+                                                               __uint_as_float(r[4 * i + 3]));
+      }
+    }
+  }
+  __syncwarp();
+  // Every CTA's partial is staged (release / acquire at cluster scope).
+  cluster_sync();
+  {
+    // CTA `rank` reduces rows [r0, r0 + rows) of the tile over the S partials.
+    constexpr int kVec = BN / 4;  // float4 per row
+    const int rows = (kProjBM + splits - 1) / splits;
+    const int r0 = rank * rows;
+    const int r1 = min(kProjBM, r0 + rows);
+    for (int item = threadIdx.x; item < (r1 - r0) * kVec; item += kProjThreads) {
+      const int row = r0 + item / kVec;
+      const int c = (item % kVec) * 4;
+      const float* src = part + row * S::kPartStride + c;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q = 0; q < splits; ++q) {
+        const float4 w = ld_cluster_f4(map_to_rank(src, static_cast<uint32_t>(q)));
+        v.x += w.x;
+        v.y += w.y;
+        v.z += w.z;
+        v.w += w.w;
+      }
+      const int grow = m0 + row;
+      const int n = n0 + c;
+      if (grow < M && n < Nout) {
+        if (bias != nullptr) {
+          v.x += bias[n];
+          v.y += bias[n + 1];
+          v.z += bias[n + 2];
+          v.w += bias[n + 3];
+        }
+        if constexpr (kOutBf16) {
+          uint2* dst = reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(y) + static_cast<size_t>(grow) * Nout + n);
+          *dst = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+        } else {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(y) + static_cast<size_t>(grow) * Nout + n);
+          if (accumulate) {
+            const float4 old = *dst;
+            v.x += old.x;
+            v.y += old.y;
+            v.z += old.z;
+            v.w += old.w;
+          }
+          *dst = v;
+        }
+      }
+    }
+  }
+  // No CTA leaves (and frees its shared memory) while another still reads it.
+  cluster_sync();
+
+  // ---- teardown: every MMA the issuer started has finished -----------------
+  if (threadIdx.x == 32) mbar_drain(&mma_done, 0);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 }  // namespace sqa

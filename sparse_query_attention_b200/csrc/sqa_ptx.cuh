@@ -338,8 +338,14 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
 }
-// Arrive-release / wait-acquire on the cluster barrier: every thread of both
-// CTAs of the pair must reach it.
+// Number of CTAs in this CTA's cluster.
+__device__ __forceinline__ uint32_t cluster_num_ctas() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+// Arrive-release / wait-acquire on the cluster barrier: every thread of every
+// CTA of the cluster must reach it (warp-converged: the .aligned forms).
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -349,6 +355,16 @@ __device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
   return r;
+}
+// 16-byte load from the shared memory of any CTA of the cluster
+// (shared::cluster address from map_to_rank).
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t cluster_addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(cluster_addr)
+               : "memory");
+  return v;
 }
 // Arrive on an mbarrier in another CTA of the cluster (shared::cluster address).
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {

@@ -66,6 +66,43 @@ def test_gemm_accumulate(sqa, M, N, K):
     assert_close(f64(c), f64(c0) + f64(a) @ f64(b), "C + A B")
 
 
+@pytest.mark.parametrize("a_mn,b_mn,M,N,K,out,with_bias,acc", [
+    (True, True, 256, 256, 16384, "f32", False, False),   # d[Wq; Wk; Wv] = dQKV^T X at the layer's shape
+    (True, True, 256, 128, 16384, "f32", False, True),    # dWo = dY^T O, accumulated into C
+    (False, False, 384, 48, 8208, "bf16", True, False),   # K-contiguous; ragged N (64-wide tile) and K
+    (False, True, 200, 16, 4112, "f32", True, False),     # ragged M, N = 16 in a 64-wide tile
+    (True, False, 128, 32, 2048, "bf16", False, False),   # 32-wide tile (K-contiguous B, N <= 32)
+    (True, True, 768, 256, 16384, "f32", False, False),   # 24 tiles: clusters smaller than eight
+])
+def test_gemm_split_k(sqa, a_mn, b_mn, M, N, K, out, with_bias, acc):
+    """Products with few output tiles and a long K, which split K over a
+    cluster and sum the partial tiles through distributed shared memory:
+    parity with the oracle (bias, accumulate, bf16 output), and the same bits
+    on a second run (the partials are summed in a fixed order)."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed(M + 5 * N + 3 * K)
+    a = _bf16((K, M) if a_mn else (M, K), g)
+    b = _bf16((K, N) if b_mn else (N, K), g, 0.02)
+    bias = torch.randn((N,), generator=g, device="cuda") if with_bias else None
+    c0 = torch.randn((M, N), generator=g, device="cuda")
+    la = sqa.SQA_MN_CONTIGUOUS if a_mn else sqa.SQA_K_CONTIGUOUS
+    lb = sqa.SQA_MN_CONTIGUOUS if b_mn else sqa.SQA_K_CONTIGUOUS
+    dt, tdt = (sqa.SQA_DT_BF16, torch.bfloat16) if out == "bf16" else (sqa.SQA_DT_F32, torch.float32)
+    runs = []
+    for _ in range(2):
+        c = c0.clone() if acc else torch.empty((M, N), dtype=tdt, device="cuda")
+        sqa.sqa_gemm(a, la, b, lb, bias, c, dt, acc, M, N, K)
+        runs.append(c)
+    sqa.sqa_device_status()
+    A = f64(a).T if a_mn else f64(a)
+    Bm = f64(b).T if b_mn else f64(b)
+    want = projection(A, Bm, None if bias is None else f64(bias))
+    if acc:
+        want = want + f64(c0)
+    assert_close(f64(runs[0]), want, "C")
+    assert torch.equal(runs[0], runs[1]), "split-K result differs between two runs"
+
+
 VARIANTS = {"GQA": (16, 4), "SQA": (8, 4), "sSQA": (8, 8), "xSQA": (4, 4), "xSMQA": (4, 1)}
 
 

@@ -58,7 +58,7 @@ def test_proj_bias_and_bf16(sqa):
 
 
 @pytest.mark.parametrize("M,K,Nout,bf16_out", [(4100, 528, 2320, True), (4100, 528, 2320, False),
-                                                (2048, 4096, 512, True)])
+                                                (8200, 1008, 784, True)])
 def test_proj_pair_tiles(sqa, M, K, Nout, bf16_out):
     """Products large enough to run on CTA pairs (256 x 256 tiles, two SMs per
     tile): ragged M, Nout and K (M not a multiple of 256, Nout of 256, K of
