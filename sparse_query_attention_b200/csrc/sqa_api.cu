@@ -86,6 +86,63 @@ sqa_status_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
 }
 
+// launch_k for a grid of thread-block clusters of `cluster_x` CTAs along x.
+template <typename... KArgs, typename... Args>
+sqa_status_t launch_k_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster_x;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
+}
+
+// How many clusters of `cluster` CTAs of `kern` (`threads` per CTA, `smem`
+// bytes of dynamic shared memory, already allowed by cudaFuncSetAttribute)
+// the current device runs at once.  Queried once per device, kernel and
+// cluster size; 0 when the query fails.
+int max_active_clusters(const void* kern, int cluster, int threads, int smem) {
+  struct Entry {
+    int dev;
+    const void* kern;
+    int cluster;
+    int n;
+  };
+  static Entry cache[128];
+  static int used = 0;
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].dev == dev && cache[i].kern == kern && cache[i].cluster == cluster) return cache[i].n;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(cluster * 64);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 0) n = 0;
+  if (used < 128) cache[used++] = {dev, kern, cluster, n};
+  return n;
+}
+
 bool supported_d(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 
 // Streaming multiprocessors of the current device (looked up per call; the
@@ -402,6 +459,7 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
   p.win_l = a.win_l;
   p.win_r = a.win_r;
   p.longest_first = a.longest_first;
+  p.kv_splits = 1;
   p.scale = a.scale;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.ld_dq = static_cast<int>(a.ld_dq);
@@ -437,9 +495,30 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
     constexpr int smem = sqa::DkdvCfg<D>::kSmemBytes;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return SQA_ERR_CUDA;
-    dim3 grid((Nkv + 127) / 128, H_kv, B);
-    s = launch_k(kern, grid, dim3(sqa::kBwdThreads), smem, st, m_k128, m_v128, m_q64, m_do64, m_l2, m_ds, p);
+    // Unmasked problems whose key tiles leave SMs idle (cross / memory
+    // attention over a short key sequence) split each tile's steps over a
+    // cluster of 2, 4 or 8 CTAs: the largest split for which every cluster
+    // runs at once and each CTA keeps at least 8 of the tile's steps.  A grid
+    // that already fills the SMs is left whole (more, shorter CTAs in several
+    // waves measured no faster).
+    const long long units = static_cast<long long>((Nkv + 127) / 128) * H_kv * B;
+    const long long n_all = static_cast<long long>(G) * ((N + 63) / 64);
+    int splits = 1;
+    if (!a.masked && !a.longest_first) {
+      for (int c = 2; c <= 8; c *= 2) {
+        if (n_all < 8LL * c) break;
+        if (units > max_active_clusters(reinterpret_cast<const void*>(kern), c, sqa::kBwdThreads, smem)) break;
+        splits = c;
+      }
+    }
+    p.kv_splits = splits;
+    dim3 grid(static_cast<unsigned>(((Nkv + 127) / 128) * splits), H_kv, B);
+    s = splits > 1 ? launch_k_cluster(kern, grid, dim3(sqa::kBwdThreads), smem, st, splits, m_k128, m_v128, m_q64,
+                                      m_do64, m_l2, m_ds, p)
+                   : launch_k(kern, grid, dim3(sqa::kBwdThreads), smem, st, m_k128, m_v128, m_q64, m_do64, m_l2,
+                              m_ds, p);
     if (s != SQA_OK) return s;
+    p.kv_splits = 1;
   }
   // 3. dQ (Q-outer).
   {
@@ -555,34 +634,16 @@ sqa_status_t launch_gemm_pair(const CUtensorMap& ma, const CUtensorMap& mb, cons
 // Split K over clusters (proj_gemm_splitk_kernel): for products with few
 // output tiles and a long K.  Clusters of 8, 4 or 2 CTAs, the largest for
 // which one cluster per output tile fits on the device at once and each CTA
-// keeps at least four K blocks; 0 when none does.  How many clusters of a
-// size fit is queried once per device and size.
+// keeps at least four K blocks; 0 when none does.
 template <int BN, bool kBf16, bool kAMN, bool kBMN>
 int gemm_split_count(long long tiles, int num_kb) {
-  static int max_clusters[kMaxDevices][3] = {};  // 0: not queried yet; -1: query failed
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
   auto kern = sqa::proj_gemm_splitk_kernel<BN, kBf16, kAMN, kBMN>;
   constexpr int smem = sqa::SplitSmem<BN>::kDynamicBytes;
-  for (int splits = 8, slot = 2; splits >= 2; splits /= 2, --slot) {
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 0;
+  for (int splits = 8; splits >= 2; splits /= 2) {
     if (num_kb < 4 * splits) continue;
-    if (max_clusters[dev][slot] == 0) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 0;
-      cudaLaunchConfig_t cfg = {};
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = splits;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.gridDim = dim3(splits * 64);
-      cfg.blockDim = dim3(sqa::kProjThreads);
-      cfg.dynamicSmemBytes = smem;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int n = 0;
-      max_clusters[dev][slot] = cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0 ? n : -1;
-    }
-    if (tiles <= max_clusters[dev][slot]) return splits;
+    if (tiles <= max_active_clusters(reinterpret_cast<const void*>(kern), splits, sqa::kProjThreads, smem))
+      return splits;
   }
   return 0;
 }

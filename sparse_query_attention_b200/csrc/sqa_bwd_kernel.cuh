@@ -112,6 +112,17 @@ __device__ __forceinline__ void store16<__nv_bfloat16>(__nv_bfloat16* dst, const
                      pack_bf16x2(v[14], v[15]));
 }
 
+template <typename T>
+__device__ __forceinline__ void store4(T* dst, float4 v);
+template <>
+__device__ __forceinline__ void store4<float>(float* dst, float4 v) {
+  *reinterpret_cast<float4*>(dst) = v;
+}
+template <>
+__device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* dst, float4 v) {
+  *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+}
+
 // Swizzled-tile geometry shared by the backward kernels: R rows of D bf16,
 // stored as D/64 column chunks of R rows x (up to) 128 bytes.
 template <int D, int R>
@@ -149,6 +160,7 @@ struct BwdParams {
   int masked;                   // band mask active (causal or sliding window)
   int win_l, win_r;             // band: t - win_l <= u <= t + win_r (both <= N)
   int longest_first;            // causal: hand out the longest tiles first over the whole grid
+  int kv_splits;                // dK/dV: CTAs (a cluster) sharing one key tile's steps; 1 = none
   float scale;
   float scale_log2;
 };
@@ -193,6 +205,9 @@ struct DkdvCfg {
   __device__ static constexpr uint32_t col_dp(int b) { return 64u + 128u * b; }
   static constexpr uint32_t kColDV = 128 * kBufs, kColDK = 128 * kBufs + D;
   static_assert(kColDK + D <= 512, "TMEM columns");
+  // Split over a cluster: partial dV and dK rows staged over the ring.
+  static constexpr int kPartStride = D + 4;  // floats per row; the pad spreads rows over the banks
+  static_assert(2 * 128 * kPartStride * 4 <= kStages * kStageBytes, "partial dV / dK fit over the ring");
 };
 
 // Splits v into three bf16 parts whose sum is v to about 2^-24 relative.
@@ -235,7 +250,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int lane = threadIdx.x & 31;
   // Causal: key tile 0 sees every query, so ascending tiles are longest first.
   const BlockUnit u = block_unit(p.longest_first);
-  const int kt = u.x;  // key tile
+  // Unmasked problems with few key tiles (cross / memory attention over a
+  // short key sequence) split each key tile's steps over a cluster of
+  // p.kv_splits CTAs: CTA `rank` takes a contiguous share of the
+  // (query head, query sub-tile) steps, and the partial dK / dV are summed
+  // through distributed shared memory at the end.
+  const int splits = p.kv_splits;
+  const int rank = splits > 1 ? static_cast<int>(cluster_rank()) : 0;
+  const int kt = splits > 1 ? u.x / splits : u.x;  // key tile
   const int j = u.y;
   const int b = u.z;
   const int key0 = kt * 128;
@@ -245,7 +267,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int q_hi = p.masked ? min(p.N, key0 + 128 + p.win_l) : p.N;
   const int qs_begin = q_lo / 64;
   const int per_head = max(0, (q_hi + 63) / 64 - qs_begin);
-  const int n_steps = p.G * per_head;
+  const int n_all = p.G * per_head;  // steps of this key tile; this CTA runs [s_begin, s_begin + n_steps)
+  const int s_begin = static_cast<int>(static_cast<long long>(n_all) * rank / splits);
+  const int n_steps = static_cast<int>(static_cast<long long>(n_all) * (rank + 1) / splits) - s_begin;
 
   if (threadIdx.x == 0) {
     mbar_init(&kv_full, 1);
@@ -329,8 +353,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (; s < n_steps; ++s) {
         const int st = s % C::kStages;
         if (s >= C::kStages && !mbar_wait(&st_empty[st], ((s / C::kStages) - 1) & 1, &abort_flag)) break;
-        const int h = j * p.G + s / per_head;
-        const int q0 = (qs_begin + s % per_head) * 64;
+        const int h = j * p.G + (s_begin + s) / per_head;
+        const int q0 = (qs_begin + (s_begin + s) % per_head) * 64;
         uint8_t* dst = stages + st * C::kStageBytes;
         mbar_arrive_expect_tx(&st_full[st], 2 * QT::kBytes + 512);
         for (int c = 0; c < QT::kChunks; ++c) {
@@ -451,7 +475,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint8_t* stat = stages + (s % C::kStages) * C::kStageBytes + 2 * QT::kBytes;
       const float* l2 = reinterpret_cast<const float*>(stat + C::kStatLse);
       const float* dd = reinterpret_cast<const float*>(stat + C::kStatD);
-      const int q0 = (qs_begin + s % per_head) * 64;
+      const int q0 = (qs_begin + (s_begin + s) % per_head) * 64;
       // Query column c (token q0 + c) contributes iff q0 + c < N and key u
       // is inside its band: u - win_r <= q0 + c <= u + win_l.  Full tiles
       // skip the per-element test.
@@ -559,6 +583,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (lane == 0) mbar_arrive(&p_ready[buf]);
     }
     // ---------------- epilogue: group 0 writes dV, group 1 writes dK --------
+    // With a split, each CTA stages its partial rows over the operand ring
+    // (idle once mma_done has fired: every copy into it was consumed by an
+    // MMA, and the statistics warp finished before the last one).
     if (ok) ok = mbar_wait(&mma_done, 0, &abort_flag);
     if (ok) {
       tc_fence_after();
@@ -567,6 +594,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float mult = grp == 0 ? 1.f : p.scale;
       GradT* dst = static_cast<GradT*>(grp == 0 ? p.dv : p.dk) +
                    (static_cast<size_t>(b) * p.Nkv + (valid ? u : 0)) * p.ld_dkv + static_cast<size_t>(j) * D;
+      float* part = reinterpret_cast<float*>(stages) + (grp * 128 + r) * C::kPartStride;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 16) {
         uint32_t rr[16];
@@ -575,12 +603,51 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         float v[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) v[c] = (n_steps > 0 ? __uint_as_float(rr[c]) : 0.f) * mult;
-        if (valid) store16<GradT>(dst + c0, v);
+        if (splits > 1) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            reinterpret_cast<float4*>(part + c0)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        } else if (valid) {
+          store16<GradT>(dst + c0, v);
+        }
       }
     }
   }
 
   __syncwarp();
+  if (splits > 1) {
+    // Every CTA of the cluster has staged its partial dV and dK (release /
+    // acquire at cluster scope).  CTA `rank` sums rows [r0, r1) of both over
+    // the cluster, in rank order, and writes them; the second barrier keeps
+    // every CTA's shared memory alive until all reads are done.
+    cluster_sync();
+    constexpr int kVec = D / 4;  // float4 per row
+    const int rows = (128 + splits - 1) / splits;
+    const int r0 = rank * rows;
+    const int nr = max(0, min(128, r0 + rows) - r0);
+    const float* part = reinterpret_cast<const float*>(stages);
+    for (int item = threadIdx.x; item < 2 * nr * kVec; item += kBwdThreads) {
+      const int which = item / (nr * kVec);  // 0: dV, 1: dK
+      const int rem = item - which * nr * kVec;
+      const int row = r0 + rem / kVec;
+      const int c = (rem % kVec) * 4;
+      const float* src = part + (which * 128 + row) * C::kPartStride + c;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q = 0; q < splits; ++q) {
+        const float4 w = ld_cluster_f4(map_to_rank(src, static_cast<uint32_t>(q)));
+        acc.x += w.x;
+        acc.y += w.y;
+        acc.z += w.z;
+        acc.w += w.w;
+      }
+      const int tok = key0 + row;
+      if (tok < p.Nkv)
+        store4<GradT>(static_cast<GradT*>(which == 0 ? p.dv : p.dk) +
+                          (static_cast<size_t>(b) * p.Nkv + tok) * p.ld_dkv + static_cast<size_t>(j) * D + c,
+                      acc);
+    }
+    cluster_sync();
+  }
   if (threadIdx.x == 32) mbar_drain(&mma_done, 0);
   tc_fence_before();
   __syncthreads();

@@ -111,3 +111,33 @@ def test_cross_equal_lengths_match_self_attention(sqa):
                         1 / math.sqrt(64))
     torch.cuda.synchronize()
     assert torch.equal(o, o2) and torch.equal(lse, lse2)
+
+
+# Few key tiles against many queries: each key tile's dK/dV steps are split
+# over a cluster of 2, 4 or 8 CTAs and the partial dK/dV summed through
+# distributed shared memory.  Ragged key lengths, G = 3 (the CTAs' shares of
+# the steps end inside a head), d from 16 to 128, non-causal self-attention
+# (N_q = N_kv), and the same bits on a second run (fixed summation order).
+SPLIT_SHAPES = [
+    (1, 4096, 1024, 8, 4, 128),   # 32 key tiles x heads: clusters of 4
+    (1, 1000, 300, 6, 2, 64),     # G = 3, shares cross head boundaries
+    (2, 2048, 77, 4, 4, 32),      # one ragged key tile per head
+    (1, 3000, 200, 4, 1, 16),     # clusters of 8
+    (1, 2048, 2048, 8, 4, 64),    # non-causal self-attention: clusters of 2
+]
+
+
+@pytest.mark.parametrize("B,N_q,N_kv,H_q,H_kv,d", SPLIT_SHAPES)
+def test_cross_backward_split_key_tiles(sqa, B, N_q, N_kv, H_q, H_kv, d):
+    x = cross_attention_inputs(B, N_q, N_kv, H_q, H_kv, d, seed=N_q * 41 + N_kv, with_dout=True, device="cuda")
+    o, lse = _fwd(sqa, x)
+    g1 = _bwd(sqa, x, o, lse)
+    g2 = _bwd(sqa, x, o, lse)
+    torch.cuda.synchronize()
+    sqa.sqa_device_status()
+    rq, rk, rv = attention_backward(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(x["do"]), False, 1 / math.sqrt(d))
+    assert_close(f64(g1[0]), rq, "dQ")
+    assert_close(f64(g1[1]), rk, "dK")
+    assert_close(f64(g1[2]), rv, "dV")
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b), "gradients differ between two runs"
