@@ -950,6 +950,7 @@ def run_sqa(args):
                      "frac": achieved / peak, "traffic": traffic, "peak_source": f"{peak_kind} bf16 burst"},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps, "mode": "pipelined: copies of neighbouring steps overlap the kernel",
+                "ms_per_step": e2e_ms / e2e_steps, "kernel_ms_per_step": ms_per_step,
                 "serial_value": e2e_serial},
         "gpu_launches": args.steps,
         "variants": variants,
