@@ -304,6 +304,7 @@ sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* ou
   p.longest_first = a.longest_first;
   p.tblk0 = 0;
   p.wait_at_exit = 0;
+  p.kv_splits = 1;
   p.out_bf16 = out_bf16;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const long long gy = static_cast<long long>(H_kv) * p.n_sub;
@@ -330,6 +331,32 @@ sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* ou
     // ran 2 % slower split), so masked problems keep the two-tile grid.
     const int sms = num_sms();
     if (sms <= 0) return SQA_ERR_CUDA;
+    // Few query tiles against many keys (unmasked: cross attention from a
+    // short query sequence, or small batches): split every token block's key
+    // range over a cluster of 2, 4 or 8 two-tile CTAs, the largest for which
+    // all clusters run at once and each CTA keeps at least four key blocks;
+    // the CTAs merge their rows' partial results in distributed shared memory.
+    // (A cluster's CTAs are consecutive along x, so the grid keeps its plain
+    // order: unmasked problems never take the longest-first order.)
+    if (!a.masked && !a.longest_first) {
+      auto kern = sqa::sqa_fwd_kernel<D, true>;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+        return SQA_ERR_CUDA;
+      const long long units = static_cast<long long>(p.n_tblk) * gy * B;
+      const int nb = (Nkv + 127) / 128;
+      int splits = 1;
+      for (int c = 2; c <= 8; c *= 2) {
+        if (nb < 4 * c) break;
+        if (units > max_active_clusters(reinterpret_cast<const void*>(kern), c, sqa::kFwdThreads, C::kSmemBytes))
+          break;
+        splits = c;
+      }
+      if (splits > 1) {
+        p.kv_splits = splits;
+        const dim3 grid_c(static_cast<unsigned>(p.n_tblk * splits), static_cast<unsigned>(gy), B);
+        return launch_k_cluster(kern, grid_c, dim3(sqa::kFwdThreads), C::kSmemBytes, st, splits, mq, mk, mv, p);
+      }
+    }
     constexpr double kSplitWave = 0.55;
     const long long yz = gy * B;
     const int n_tiles = (N + T - 1) / T;

@@ -53,6 +53,12 @@ struct FwdCfg {
   static constexpr int kSmemBytes = kQBytes + kSlots * kTileBytes + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
+  // Key split over a cluster: per row of both tiles, the unnormalised O
+  // (padded rows, spread over the banks) and then (running max, sum) as one
+  // 16-byte slot, staged over Q and the ring.
+  static constexpr int kPartStride = D + 4;         // floats per staged O row
+  static constexpr int kPartMl = 256 * kPartStride;  // float offset of the (m, l) slots
+  static_assert(kPartMl * 4 + 256 * 16 <= kQBytes + kSlots * kTileBytes, "staged rows fit over Q and the ring");
 };
 
 struct FwdParams {
@@ -67,6 +73,7 @@ struct FwdParams {
   int longest_first;  // schedule token blocks from the last one
   int tblk0;          // first token block of this launch (a problem may be split over two launches)
   int wait_at_exit;   // second launch of a split problem: wait for the previous grid only before exiting
+  int kv_splits;      // two-tile kernel: CTAs (a cluster) sharing one token block's key range; 1 = none
   int out_bf16;
   float scale_log2;  // scale * log2(e)
 };
@@ -79,7 +86,9 @@ static_assert(kFwdRegsLow * 128 + kFwdRegsHigh * 256 <= kFwdRegsLaunch * kFwdThr
               "register split exceeds the launch pool");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only past 2^8 growth
 
-template <int D>
+// kKvSplit: the instantiation launched in clusters that split the key range
+// (p.kv_splits > 1); the other one carries none of that code.
+template <int D, bool kKvSplit = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     sqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -105,7 +114,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   // ---- work unit -----------------------------------------------------------
   const int T = 128 >> p.log2g;  // tokens per tile
   const BlockUnit u = block_unit(p.longest_first);
-  const int tblk = p.tblk0 + (p.longest_first ? (p.n_tblk - 1 - u.x) : u.x);
+  // Few query tiles against many keys (unmasked): the key blocks of a token
+  // block are split over a cluster of p.kv_splits CTAs, CTA `rank` taking a
+  // contiguous share; each row's partial O, running max and sum are merged
+  // through distributed shared memory at the end.
+  const int splits = kKvSplit ? p.kv_splits : 1;
+  const int rank = kKvSplit ? static_cast<int>(cluster_rank()) : 0;
+  const int ux = kKvSplit ? u.x / splits : u.x;
+  const int tblk = p.tblk0 + (p.longest_first ? (p.n_tblk - 1 - ux) : ux);
   const int j = u.y / p.n_sub;
   const int sub = u.y % p.n_sub;
   const int b = u.z;
@@ -124,6 +140,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int hi = p.masked ? min(p.Nkv, tmax + p.win_r + 1) : p.Nkv;
     kv_lo[t] = lo / 128;
     kv_hi[t] = (hi + 127) / 128;
+  }
+  if constexpr (kKvSplit) {  // unmasked: both tiles see every key block
+    const int nb = (p.Nkv + 127) / 128;
+    kv_lo[0] = kv_lo[1] = static_cast<int>(static_cast<long long>(nb) * rank / splits);
+    kv_hi[0] = kv_hi[1] = static_cast<int>(static_cast<long long>(nb) * (rank + 1) / splits);
   }
   const int kv_begin = kv_lo[0];
   if (t0 + T >= p.N) kv_lo[1] = kv_hi[1] = kv_begin;  // tile 1 holds no token
@@ -428,7 +449,28 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     // Epilogue: O / l and LSE once the last PV of this tile has landed.
     if (ok) ok = mbar_wait(&o_done[t], 0, &abort_flag);  // committed once, after the last PV
-    if (ok) {
+    if constexpr (kKvSplit) {
+      // Stage the row's unnormalised O and its (running max, sum) over Q and
+      // the ring, once no MMA of either tile reads them any more.
+      if (ok) ok = mbar_wait(&mma_done, 0, &abort_flag);
+      if (ok) {
+        tc_fence_after();
+        float* po = reinterpret_cast<float*>(smem) + (t * 128 + r) * C::kPartStride;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 16) {
+          uint32_t orr[16];
+          tmem_ld16(o_addr + c0, orr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            reinterpret_cast<float4*>(po + c0)[q4] =
+                make_float4(__uint_as_float(orr[4 * q4]), __uint_as_float(orr[4 * q4 + 1]),
+                            __uint_as_float(orr[4 * q4 + 2]), __uint_as_float(orr[4 * q4 + 3]));
+        }
+        reinterpret_cast<float4*>(reinterpret_cast<float*>(smem) + C::kPartMl)[t * 128 + r] =
+            make_float4(m_used, l_sum, 0.f, 0.f);
+      }
+    } else if (ok) {
       tc_fence_after();
       const bool valid = tok < p.N;
       const float inv_l = 1.f / l_sum;
@@ -461,8 +503,59 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
   }
 
-  // ---- teardown ------------------------------------------------------------
   __syncwarp();
+  if constexpr (kKvSplit) {
+    // Every CTA of the cluster has staged its rows (release / acquire at
+    // cluster scope).  CTA `rank` merges rows [R0, R0 + nr) of the 256 (two
+    // tiles) over the cluster in rank order:
+    //   m = max_q m_q,  w_q = 2^(m_q - m),  l = sum_q w_q l_q,
+    //   O = sum_q w_q O_q / l,  LSE = (m + log2 l) ln 2,
+    // the merge a split of the key range admits; the second barrier keeps
+    // every CTA's shared memory alive until all reads are done.
+    cluster_sync();
+    constexpr int kVec = D / 4;  // float4 per row
+    const float* po = reinterpret_cast<const float*>(smem);
+    const float4* pml = reinterpret_cast<const float4*>(po + C::kPartMl);
+    const int rows = (256 + splits - 1) / splits;
+    const int R0 = rank * rows;
+    const int nr = max(0, min(256, R0 + rows) - R0);
+    for (int item = threadIdx.x; item < nr * kVec; item += kFwdThreads) {
+      const int R = R0 + item / kVec;
+      const int c = (item % kVec) * 4;
+      const int rr = R & 127;
+      const int tok_r = t0 + (R >> 7) * T + (rr >> p.log2g);
+      if (tok_r >= p.N) continue;
+      const int head_r = h0 + (rr & (p.g - 1));
+      float m = -INFINITY;
+      for (int q = 0; q < splits; ++q) m = fmaxf(m, ld_cluster_f4(map_to_rank(pml + R, static_cast<uint32_t>(q))).x);
+      float l = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q = 0; q < splits; ++q) {
+        const float4 ml = ld_cluster_f4(map_to_rank(pml + R, static_cast<uint32_t>(q)));
+        const float w = ml.x == -INFINITY ? 0.f : ex2_approx(ml.x - m);
+        l += ml.y * w;
+        const float4 o = ld_cluster_f4(map_to_rank(po + R * C::kPartStride + c, static_cast<uint32_t>(q)));
+        acc.x += w * o.x;
+        acc.y += w * o.y;
+        acc.z += w * o.z;
+        acc.w += w * o.w;
+      }
+      const float inv_l = 1.f / l;
+      const size_t off = ((static_cast<size_t>(b) * p.N + tok_r) * p.H_q + head_r) * D + c;
+      if (p.out_bf16) {
+        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + off) =
+            make_uint2(pack_bf16x2(acc.x * inv_l, acc.y * inv_l), pack_bf16x2(acc.z * inv_l, acc.w * inv_l));
+      } else {
+        *reinterpret_cast<float4*>(static_cast<float*>(p.out) + off) =
+            make_float4(acc.x * inv_l, acc.y * inv_l, acc.z * inv_l, acc.w * inv_l);
+      }
+      if (c == 0 && p.lse != nullptr)
+        p.lse[(static_cast<size_t>(b) * p.H_q + head_r) * p.N + tok_r] = (m + __log2f(l)) * 0.69314718055994531f;
+    }
+    cluster_sync();
+  }
+
+  // ---- teardown ------------------------------------------------------------
   if (threadIdx.x == 32) mbar_drain(&mma_done, 0);  // every issued MMA has finished
   tc_fence_before();
   __syncthreads();

@@ -141,3 +141,31 @@ def test_cross_backward_split_key_tiles(sqa, B, N_q, N_kv, H_q, H_kv, d):
     assert_close(f64(g1[2]), rv, "dV")
     for a, b in zip(g1, g2):
         assert torch.equal(a, b), "gradients differ between two runs"
+
+
+# Few query tiles against many keys (d = 128, unmasked): every token block's
+# key range is split over a cluster of 2, 4 or 8 CTAs and the rows' partial
+# O, running max and sum merged through distributed shared memory.  Ragged
+# N_q (a block whose second tile is partly or wholly past N) and N_kv, G = 3
+# (one head per tile row group), fp32 and bf16 outputs with the LSE, and the
+# same bits on a second run.
+FWD_SPLIT_SHAPES = [
+    (1, 300, 5000, 8, 4, torch.float32),    # clusters of 8
+    (2, 129, 2048, 4, 4, torch.bfloat16),   # clusters of 4, one token in the second tile
+    (1, 64, 1000, 6, 2, torch.float32),     # G = 3, clusters of 2
+    (1, 1024, 1024, 8, 4, torch.bfloat16),  # non-causal self-attention shape
+]
+
+
+@pytest.mark.parametrize("B,N_q,N_kv,H_q,H_kv,odt", FWD_SPLIT_SHAPES)
+def test_cross_forward_split_key_range(sqa, B, N_q, N_kv, H_q, H_kv, odt):
+    d = 128
+    x = cross_attention_inputs(B, N_q, N_kv, H_q, H_kv, d, seed=N_q * 43 + N_kv, device="cuda")
+    o1, l1 = _fwd(sqa, x, out_dtype=odt)
+    o2, l2 = _fwd(sqa, x, out_dtype=odt)
+    torch.cuda.synchronize()
+    sqa.sqa_device_status()
+    ro, rl = attention_forward(f64(x["q"]), f64(x["k"]), f64(x["v"]), False, 1 / math.sqrt(d))
+    assert_close(f64(o1), ro, "O")
+    assert_close(f64(l1), rl, "LSE")
+    assert torch.equal(o1, o2) and torch.equal(l1, l2), "forward differs between two runs"
