@@ -527,21 +527,25 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
     // cluster of 2, 4 or 8 CTAs: the largest split for which every cluster
     // runs at once and each CTA keeps at least 8 of the tile's steps.  A grid
     // that already fills the SMs is left whole (more, shorter CTAs in several
-    // waves measured no faster).
+    // waves measured no faster).  The split is an instantiation of its own
+    // (with the statistics folded), so the unsplit kernel keeps its code.
     const long long units = static_cast<long long>((Nkv + 127) / 128) * H_kv * B;
     const long long n_all = static_cast<long long>(G) * ((N + 63) / 64);
     int splits = 1;
-    if (!a.masked && !a.longest_first) {
+    if (fold && !a.masked && !a.longest_first) {
+      auto kern_s = sqa::bwd_dkdv_kernel<D, GradT, true, true>;
+      if (cudaFuncSetAttribute(kern_s, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return SQA_ERR_CUDA;
       for (int c = 2; c <= 8; c *= 2) {
         if (n_all < 8LL * c) break;
-        if (units > max_active_clusters(reinterpret_cast<const void*>(kern), c, sqa::kBwdThreads, smem)) break;
+        if (units > max_active_clusters(reinterpret_cast<const void*>(kern_s), c, sqa::kBwdThreads, smem)) break;
         splits = c;
       }
     }
     p.kv_splits = splits;
     dim3 grid(static_cast<unsigned>(((Nkv + 127) / 128) * splits), H_kv, B);
-    s = splits > 1 ? launch_k_cluster(kern, grid, dim3(sqa::kBwdThreads), smem, st, splits, m_k128, m_v128, m_q64,
-                                      m_do64, m_l2, m_ds, p)
+    s = splits > 1 ? launch_k_cluster(sqa::bwd_dkdv_kernel<D, GradT, true, true>, grid, dim3(sqa::kBwdThreads), smem,
+                                      st, splits, m_k128, m_v128, m_q64, m_do64, m_l2, m_ds, p)
                    : launch_k(kern, grid, dim3(sqa::kBwdThreads), smem, st, m_k128, m_v128, m_q64, m_do64, m_l2,
                               m_ds, p);
     if (s != SQA_OK) return s;

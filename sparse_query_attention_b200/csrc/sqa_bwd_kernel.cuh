@@ -220,7 +220,9 @@ __device__ __forceinline__ void split3_bf16(float v, __nv_bfloat16& h, __nv_bflo
 
 // kAug: statistics folded into the score MMAs (needs a scale with a finite
 // 1 / (scale log2 e)); otherwise the softmax warps read them per column.
-template <int D, typename GradT, bool kAug>
+// kKvSplit: the instantiation launched in clusters that split each key
+// tile's steps (p.kv_splits > 1); the other one carries none of that code.
+template <int D, typename GradT, bool kAug, bool kKvSplit = false>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -255,9 +257,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // p.kv_splits CTAs: CTA `rank` takes a contiguous share of the
   // (query head, query sub-tile) steps, and the partial dK / dV are summed
   // through distributed shared memory at the end.
-  const int splits = p.kv_splits;
-  const int rank = splits > 1 ? static_cast<int>(cluster_rank()) : 0;
-  const int kt = splits > 1 ? u.x / splits : u.x;  // key tile
+  const int splits = kKvSplit ? p.kv_splits : 1;
+  const int rank = kKvSplit ? static_cast<int>(cluster_rank()) : 0;
+  const int kt = kKvSplit ? u.x / splits : u.x;  // key tile
   const int j = u.y;
   const int b = u.z;
   const int key0 = kt * 128;
@@ -603,7 +605,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         float v[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) v[c] = (n_steps > 0 ? __uint_as_float(rr[c]) : 0.f) * mult;
-        if (splits > 1) {
+        if constexpr (kKvSplit) {
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             reinterpret_cast<float4*>(part + c0)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
@@ -615,7 +617,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 
   __syncwarp();
-  if (splits > 1) {
+  if constexpr (kKvSplit) {
     // Every CTA of the cluster has staged its partial dV and dK (release /
     // acquire at cluster scope).  CTA `rank` sums rows [r0, r1) of both over
     // the cluster, in rank order, and writes them; the second barrier keeps
