@@ -551,13 +551,32 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
     if (s != SQA_OK) return s;
     p.kv_splits = 1;
   }
-  // 3. dQ (Q-outer).
+  // 3. dQ (Q-outer).  Unmasked problems whose query tiles leave SMs idle
+  // (few queries against many keys) split each tile's key sub-tiles over a
+  // cluster of 2, 4 or 8 CTAs, as dK/dV does its steps.
   {
     auto kern = sqa::bwd_dq_kernel<D, GradT>;
     constexpr int smem = sqa::DqCfg<D>::kSmemBytes;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return SQA_ERR_CUDA;
-    dim3 grid(p.n_tblk, static_cast<unsigned>(gy), B);
+    int splits = 1;
+    if (!a.masked && !a.longest_first) {
+      auto kern_s = sqa::bwd_dq_kernel<D, GradT, true>;
+      if (cudaFuncSetAttribute(kern_s, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return SQA_ERR_CUDA;
+      const long long units = static_cast<long long>(p.n_tblk) * gy * B;
+      const long long n_all = (Nkv + 63) / 64;
+      for (int c = 2; c <= 8; c *= 2) {
+        if (n_all < 8LL * c) break;
+        if (units > max_active_clusters(reinterpret_cast<const void*>(kern_s), c, sqa::kBwdThreads, smem)) break;
+        splits = c;
+      }
+    }
+    p.kv_splits = splits;
+    dim3 grid(static_cast<unsigned>(p.n_tblk * splits), static_cast<unsigned>(gy), B);
+    if (splits > 1)
+      return launch_k_cluster(sqa::bwd_dq_kernel<D, GradT, true>, grid, dim3(sqa::kBwdThreads), smem, st, splits,
+                              m_qp, m_dop, m_k64, m_v64, p);
     return launch_k(kern, grid, dim3(sqa::kBwdThreads), smem, st, m_qp, m_dop, m_k64, m_v64, p);
   }
 }

@@ -675,9 +675,15 @@ struct DqCfg {
   __device__ static constexpr uint32_t col_dp(int b) { return 64u + 128u * b; }
   static constexpr uint32_t kColDQ = 128 * kBufs;
   static_assert(kColDQ + D <= 512, "TMEM columns");
+  // Split over a cluster: partial dQ rows staged over the ring.
+  static constexpr int kPartStride = D + 4;  // floats per row; the pad spreads rows over the banks
+  static_assert(128 * kPartStride * 4 <= kStages * kStageBytes, "partial dQ fits over the ring");
 };
 
-template <int D, typename GradT>
+// kKvSplit: the instantiation launched in clusters that split each query
+// tile's key sub-tiles (p.kv_splits > 1, unmasked problems only); the other
+// one carries none of that code.
+template <int D, typename GradT, bool kKvSplit = false>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -704,7 +710,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int lane = threadIdx.x & 31;
   const int T = 128 >> p.log2g;
   const BlockUnit u = block_unit(p.longest_first);
-  const int tblk = p.longest_first ? (p.n_tblk - 1 - u.x) : u.x;
+  const int ux = kKvSplit ? u.x / p.kv_splits : u.x;
+  const int tblk = p.longest_first ? (p.n_tblk - 1 - ux) : ux;
   const int j = u.y / p.n_sub;
   const int sub = u.y % p.n_sub;
   const int b = u.z;
@@ -715,8 +722,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // within [0, Nkv), streamed as 64-key sub-tiles from ks_begin.
   const int k_lo = p.masked ? max(0, t0 - p.win_l) : 0;
   const int k_hi = p.masked ? min(p.Nkv, last_tok + p.win_r + 1) : p.Nkv;
-  const int ks_begin = k_lo / 64;
-  const int n_steps = max(0, (k_hi + 63) / 64 - ks_begin);
+  int ks_begin = k_lo / 64;
+  int n_steps = max(0, (k_hi + 63) / 64 - ks_begin);
+  // Few query tiles against many keys: the key sub-tiles are split over a
+  // cluster of p.kv_splits CTAs (CTA `rank` takes a contiguous share) and the
+  // partial dQ rows summed through distributed shared memory at the end.
+  const int splits = kKvSplit ? p.kv_splits : 1;
+  const int rank = kKvSplit ? static_cast<int>(cluster_rank()) : 0;
+  if constexpr (kKvSplit) {
+    const int a0 = static_cast<int>(static_cast<long long>(n_steps) * rank / splits);
+    const int a1 = static_cast<int>(static_cast<long long>(n_steps) * (rank + 1) / splits);
+    ks_begin += a0;
+    n_steps = a1 - a0;
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
@@ -928,6 +946,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool valid = tok < p.N;
       GradT* dst = static_cast<GradT*>(p.dq) + (static_cast<size_t>(b) * p.N + (valid ? tok : 0)) * p.ld_dq +
                    static_cast<size_t>(head) * D;
+      // With a split, the partial row is staged over the operand ring (idle
+      // once mma_done has fired: every copy into it was consumed by an MMA).
+      float* part = reinterpret_cast<float*>(stages) + r * C::kPartStride;
       // The two groups split the columns of dQ (group 0 alone when D = 16).
       constexpr int kHalf = D >= 32 ? D / 2 : D;
 #pragma unroll 1
@@ -938,12 +959,49 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         float v[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) v[c] = (n_steps > 0 ? __uint_as_float(rr[c]) : 0.f) * p.scale;
-        if (valid) store16<GradT>(dst + c0, v);
+        if constexpr (kKvSplit) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            reinterpret_cast<float4*>(part + c0)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        } else if (valid) {
+          store16<GradT>(dst + c0, v);
+        }
       }
     }
   }
 
   __syncwarp();
+  if constexpr (kKvSplit) {
+    // Every CTA of the cluster has staged its partial dQ rows (release /
+    // acquire at cluster scope).  CTA `rank` sums rows [r0, r0 + nr) over the
+    // cluster, in rank order, and writes them; the second barrier keeps every
+    // CTA's shared memory alive until all reads are done.
+    cluster_sync();
+    constexpr int kVec = D / 4;  // float4 per row
+    const int rows = (128 + splits - 1) / splits;
+    const int r0 = rank * rows;
+    const int nr = max(0, min(128, r0 + rows) - r0);
+    const float* part = reinterpret_cast<const float*>(stages);
+    for (int item = threadIdx.x; item < nr * kVec; item += kBwdThreads) {
+      const int row = r0 + item / kVec;
+      const int c = (item % kVec) * 4;
+      const int tok_r = t0 + (row >> p.log2g);
+      if (tok_r >= p.N) continue;
+      const float* src = part + row * C::kPartStride + c;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q = 0; q < splits; ++q) {
+        const float4 w = ld_cluster_f4(map_to_rank(src, static_cast<uint32_t>(q)));
+        acc.x += w.x;
+        acc.y += w.y;
+        acc.z += w.z;
+        acc.w += w.w;
+      }
+      store4<GradT>(static_cast<GradT*>(p.dq) + (static_cast<size_t>(b) * p.N + tok_r) * p.ld_dq +
+                        static_cast<size_t>(h0 + (row & (p.g - 1))) * D + c,
+                    acc);
+    }
+    cluster_sync();
+  }
   if (threadIdx.x == 32) mbar_drain(&mma_done, 0);
   tc_fence_before();
   __syncthreads();

@@ -127,7 +127,17 @@ SPLIT_SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("B,N_q,N_kv,H_q,H_kv,d", SPLIT_SHAPES)
+# Few query tiles against many keys: each query tile's key sub-tiles are
+# split over a cluster in the dQ kernel and the partial dQ rows summed.
+DQ_SPLIT_SHAPES = [
+    (1, 300, 5000, 8, 4, 128),    # ragged N_q and N_kv
+    (2, 129, 2048, 4, 4, 64),     # a query tile with one token
+    (1, 64, 1000, 6, 2, 32),      # G = 3, clusters of 2
+    (1, 100, 3000, 4, 1, 16),     # four heads per tile (g = 4)
+]
+
+
+@pytest.mark.parametrize("B,N_q,N_kv,H_q,H_kv,d", SPLIT_SHAPES + DQ_SPLIT_SHAPES)
 def test_cross_backward_split_key_tiles(sqa, B, N_q, N_kv, H_q, H_kv, d):
     x = cross_attention_inputs(B, N_q, N_kv, H_q, H_kv, d, seed=N_q * 41 + N_kv, with_dout=True, device="cuda")
     o, lse = _fwd(sqa, x)
