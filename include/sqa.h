@@ -120,6 +120,9 @@ sqa_status_t sqa_attn_bwd(const void* q, const void* k, const void* v,
  * Otherwise as sqa_attn_fwd_ex with causal = 0: N_q, N_kv >= 1, any pair
  * (N_kv may be shorter or longer than N_q).  sqa_attn_fwd_ex(..., N, ...)
  * equals sqa_attn_fwd_cross(..., N_q = N, N_kv = N, ...) non-causal.
+ * Unmasked problems with few query tiles (d_head = 128) may run as clusters
+ * of CTAs that split the key range and merge their partial rows in a fixed
+ * order: the result does not change from run to run.
  */
 sqa_status_t sqa_attn_fwd_cross(const void* q, const void* k, const void* v, void* out,
                                 sqa_dtype_t out_dtype, float* lse,
@@ -131,7 +134,10 @@ sqa_status_t sqa_attn_fwd_cross(const void* q, const void* k, const void* v, voi
  * sqa_attn_bwd with causal = 0 and the two lengths apart: q, out, dout, dq
  * [B, N_q, H_q, d]; k, v, dk, dv [B, N_kv, H_kv, d]; lse [B, H_q, N_q].
  * The workspace is sqa_attn_bwd_workspace_size(B, N_q, H_q, H_kv, d_head)
- * bytes (it holds per-query-row values only).
+ * bytes (it holds per-query-row values only).  Unmasked problems with few key
+ * tiles (dK/dV) or few query tiles (dQ) may run as clusters of CTAs that
+ * split the other sequence and sum their partial gradients in a fixed order:
+ * the gradients do not change from run to run, and no workspace is added.
  */
 sqa_status_t sqa_attn_bwd_cross(const void* q, const void* k, const void* v,
                                 const void* out, sqa_dtype_t o_dtype,
@@ -291,6 +297,9 @@ sqa_status_t sqa_proj(const void* x, const void* w, const float* bias, void* y,
  *                        or  b[k * N + n]  (SQA_MN_CONTIGUOUS)
  * a, b bf16; c row-major [M, N] in c_dtype; bias NULL or fp32 [N].
  * accumulate != 0 adds into the existing C (fp32 C only).
+ * Products with few output tiles and a long K (weight gradients, K = tokens)
+ * split K over clusters of CTAs and sum the partial tiles in a fixed order:
+ * C does not change from run to run, and no workspace is needed.
  * Requirements: M, N, K >= 1; K % 16 == 0; N % 16 == 0; M % 16 == 0 when A
  * is MN-contiguous.  Examples (y = x W^T, x [M, K], W [N, K]):
  *   forward  y  = sqa_gemm(x, K_CONTIGUOUS, W, K_CONTIGUOUS)            (M, N, K)
