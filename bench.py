@@ -652,54 +652,67 @@ LAYER = {"B": 16, "N": 1024, "d_model": 256, "d_head": 16, "causal": True}
 LAYER_VARIANTS = {"MHA": (16, 16), "GQA": (16, 4), "SQA": (8, 4), "sSQA": (8, 8), "xSQA": (4, 4), "xSMQA": (4, 1)}
 
 
-def time_decoder_layer(sqa, torch, stream, flush, dev, reps=5):
-    """Forward and training step of the small decoder attention layer (B=16,
-    N=1024, d_model=256, d_head=16, causal), per head-count variant (median of
-    reps, L2 flushed).  The input projection is fused: one GEMM with the
-    concatenated weight [Wq; Wk; Wv] writes a packed QKV buffer that the
-    attention reads in place; the backward writes packed dQKV, so dX and
-    d[Wq; Wk; Wv] are one GEMM each.  Forward 3 launches, training step 10."""
+def decoder_layer_step(sqa, torch, stream, dev, name):
+    """The small decoder attention layer (B=16, N=1024, d_model=256,
+    d_head=16, causal) at one head-count variant: returns its forward and
+    its backward as two closures over their own buffers.  The input
+    projection is fused: one GEMM with the concatenated weight [Wq; Wk; Wv]
+    writes a packed QKV buffer that the attention reads in place; the
+    backward writes packed dQKV, so dX and d[Wq; Wk; Wv] are one GEMM each."""
     from sqa_inputs import layer_inputs
 
+    c = LAYER
+    B, N, dm, dh = c["B"], c["N"], c["d_model"], c["d_head"]
+    hq, hkv = LAYER_VARIANTS[name]
+    M = B * N
+    x = layer_inputs(B, N, dm, hq, hkv, dh, seed=1, device=dev)
+    W = (hq + 2 * hkv) * dh
+    w_qkv = torch.cat([x["wq"], x["wk"], x["wv"]], dim=0).contiguous()
+    qkv = torch.empty((M, W), dtype=torch.bfloat16, device=dev)
+    o = torch.empty((M, hq * dh), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((M, dm), dtype=torch.float32, device=dev)
+    lse = torch.empty((B, hq, N), dtype=torch.float32, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(11)
+    dy = torch.randn((M, dm), generator=gen, device=dev).to(torch.bfloat16)
+    do = torch.empty_like(o)
+    dqkv = torch.empty_like(qkv)
+    dx = torch.empty((M, dm), dtype=torch.float32, device=dev)
+    dw_qkv = torch.empty((W, dm), dtype=torch.float32, device=dev)
+    dwo = torch.empty((dm, hq * dh), dtype=torch.float32, device=dev)
+    wsb = sqa.sqa_attn_bwd_workspace_size(B, N, hq, hkv, dh)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    KC, MN, BF, F32 = sqa.SQA_K_CONTIGUOUS, sqa.SQA_MN_CONTIGUOUS, sqa.SQA_DT_BF16, sqa.SQA_DT_F32
+    sc = 1 / math.sqrt(dh)
+
+    def layer():
+        sqa.sqa_proj(x["x"], w_qkv, None, qkv, BF, M, dm, W, stream=stream)
+        sqa.sqa_attn_fwd_packed(qkv, o, BF, lse, B, N, hq, hkv, dh, True, sc, stream=stream)
+        sqa.sqa_proj(o, x["wo"], None, y, F32, M, hq * dh, dm, stream=stream)
+
+    def layer_backward():
+        sqa.sqa_gemm(dy, KC, x["wo"], MN, None, do, BF, False, M, hq * dh, dm, stream=stream)
+        sqa.sqa_gemm(dy, MN, o, MN, None, dwo, F32, False, dm, hq * dh, M, stream=stream)
+        sqa.sqa_attn_bwd_packed(qkv, o, BF, do, lse, dqkv, BF, B, N, hq, hkv, dh, True, sc, ws, wsb,
+                                stream=stream)
+        sqa.sqa_gemm(dqkv, KC, w_qkv, MN, None, dx, F32, False, M, dm, W, stream=stream)
+        sqa.sqa_gemm(dqkv, MN, x["x"], MN, None, dw_qkv, F32, False, W, dm, M, stream=stream)
+
+    return layer, layer_backward
+
+
+def time_decoder_layer(sqa, torch, stream, flush, dev, reps=5):
+    """Forward and training step of the small decoder attention layer (B=16,
+    N=1024, d_model=256, d_head=16, causal; decoder_layer_step), per
+    head-count variant (median of reps, L2 flushed).  Forward 3 launches,
+    training step 10."""
     c = LAYER
     B, N, dm, dh = c["B"], c["N"], c["d_model"], c["d_head"]
     M = B * N
     P_c = N * (N + 1) // 2
     out = {}
     for name, (hq, hkv) in LAYER_VARIANTS.items():
-        x = layer_inputs(B, N, dm, hq, hkv, dh, seed=1, device=dev)
-        W = (hq + 2 * hkv) * dh
-        w_qkv = torch.cat([x["wq"], x["wk"], x["wv"]], dim=0).contiguous()
-        qkv = torch.empty((M, W), dtype=torch.bfloat16, device=dev)
-        o = torch.empty((M, hq * dh), dtype=torch.bfloat16, device=dev)
-        y = torch.empty((M, dm), dtype=torch.float32, device=dev)
-
-        lse = torch.empty((B, hq, N), dtype=torch.float32, device=dev)
-        gen = torch.Generator(device=dev)
-        gen.manual_seed(11)
-        dy = torch.randn((M, dm), generator=gen, device=dev).to(torch.bfloat16)
-        do = torch.empty_like(o)
-        dqkv = torch.empty_like(qkv)
-        dx = torch.empty((M, dm), dtype=torch.float32, device=dev)
-        dw_qkv = torch.empty((W, dm), dtype=torch.float32, device=dev)
-        dwo = torch.empty((dm, hq * dh), dtype=torch.float32, device=dev)
-        wsb = sqa.sqa_attn_bwd_workspace_size(B, N, hq, hkv, dh)
-        ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
-        KC, MN, BF, F32 = sqa.SQA_K_CONTIGUOUS, sqa.SQA_MN_CONTIGUOUS, sqa.SQA_DT_BF16, sqa.SQA_DT_F32
-        sc = 1 / math.sqrt(dh)
-
-        def layer():
-            sqa.sqa_proj(x["x"], w_qkv, None, qkv, BF, M, dm, W, stream=stream)
-            sqa.sqa_attn_fwd_packed(qkv, o, BF, lse, B, N, hq, hkv, dh, True, sc, stream=stream)
-            sqa.sqa_proj(o, x["wo"], None, y, F32, M, hq * dh, dm, stream=stream)
-
-        def layer_backward():
-            sqa.sqa_gemm(dy, KC, x["wo"], MN, None, do, BF, False, M, hq * dh, dm, stream=stream)
-            sqa.sqa_gemm(dy, MN, o, MN, None, dwo, F32, False, dm, hq * dh, M, stream=stream)
-            sqa.sqa_attn_bwd_packed(qkv, o, BF, do, lse, dqkv, BF, B, N, hq, hkv, dh, True, sc, ws, wsb,
-                                    stream=stream)
-            sqa.sqa_gemm(dqkv, KC, w_qkv, MN, None, dx, F32, False, M, dm, W, stream=stream)
-            sqa.sqa_gemm(dqkv, MN, x["x"], MN, None, dw_qkv, F32, False, W, dm, M, stream=stream)
+        layer, layer_backward = decoder_layer_step(sqa, torch, stream, dev, name)
 
         def timed(fn):
             for _ in range(3):
@@ -1015,6 +1028,29 @@ def run_profile(args):
         for _ in range(args.steps):
             sqa.sqa_attn_decode(q, kc, vc, lens, out, sqa.SQA_DT_BF16, None, B, n_new, hq, hkv, d, L,
                                 1 / math.sqrt(d), ws if wsb else None, wsb, stream=stream)
+    elif args.profile == "layer":
+        layer, layer_backward = decoder_layer_step(sqa, torch, stream, dev, "SQA")
+        for _ in range(args.steps):
+            layer()
+            layer_backward()
+    elif args.profile == "memattn":
+        from sqa_inputs import cross_attention_inputs
+        hq, hkv, d = 8, 4, 128
+        sc = 1 / math.sqrt(d)
+        BF = sqa.SQA_DT_BF16
+        # A short key sequence (dK/dV split) and few queries (forward and dQ
+        # split), forward and backward each, bf16 in and out.
+        for Nq, Nkv in ((32768, 1024), (1024, 32768)):
+            x = cross_attention_inputs(1, Nq, Nkv, hq, hkv, d, seed=3, with_dout=True, device=dev)
+            o = torch.empty((1, Nq, hq, d), dtype=torch.bfloat16, device=dev)
+            lse = torch.empty((1, hq, Nq), dtype=torch.float32, device=dev)
+            g = [torch.empty(t.shape, dtype=torch.bfloat16, device=dev) for t in (x["q"], x["k"], x["v"])]
+            wsb = sqa.sqa_attn_bwd_workspace_size(1, Nq, hq, hkv, d)
+            ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+            for _ in range(args.steps):
+                sqa.sqa_attn_fwd_cross(x["q"], x["k"], x["v"], o, BF, lse, 1, Nq, Nkv, hq, hkv, d, sc, stream=stream)
+                sqa.sqa_attn_bwd_cross(x["q"], x["k"], x["v"], o, BF, x["do"], lse, g[0], g[1], g[2], BF, 1, Nq, Nkv,
+                                       hq, hkv, d, sc, ws, wsb, stream=stream)
     else:
         flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
         time_training_step(sqa, torch, stream, flush, dev, reps=max(1, args.steps - 3))
@@ -1030,12 +1066,15 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["sqa", "reference"], default="sqa")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["fwd", "xsqa", "mha", "gqa", "bwd", "decode", "gemm"], default=None,
+    ap.add_argument("--profile", choices=["fwd", "xsqa", "mha", "gqa", "bwd", "decode", "gemm", "layer", "memattn"],
+                    default=None,
                     help="only launch the kernels (for ncu): fwd = the bench workload's forward, "
                          "xsqa / mha / gqa = its xSQA (4,4), MHA (16,16) or GQA (16,4) variant, "
                          "gemm = the M=32768, N=K=4096 projection GEMM, "
                          "bwd = the B=4, N=8192 causal training step, decode = one SQA decode step of "
-                         "B=16 sequences x 32768 cached tokens; no timing, no JSON")
+                         "B=16 sequences x 32768 cached tokens, layer = the SQA decoder-layer training "
+                         "step (B=16, N=1024, d_model=256), memattn = SQA cross attention forward and "
+                         "backward at 32768 queries x 1024 keys and 1024 x 32768; no timing, no JSON")
     args = ap.parse_args(argv)
     if args.profile:
         return run_profile(args)
