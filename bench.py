@@ -844,7 +844,10 @@ def run_sqa(args):
     ho = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
     dsets = [tuple(torch.empty_like(t) for t in (x["q"], x["k"], x["v"])) for _ in range(2)]
     douts = [torch.empty_like(out) for _ in range(2)]
-    e2e_steps = max(10, min(args.steps, 50))
+    # A fixed 50-step window (reported as e2e.steps), whatever --steps is:
+    # the pipeline's first copy-in and last read-back are not overlapped, and
+    # over 50 steps they cost ~3 % instead of ~7 % at 20.
+    e2e_steps = 50
 
     def serial_step():
         dq_, dk_, dv_ = dsets[0]
