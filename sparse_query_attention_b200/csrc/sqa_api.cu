@@ -487,6 +487,7 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
   p.win_r = a.win_r;
   p.longest_first = a.longest_first;
   p.kv_splits = 1;
+  p.wait_at_exit = 0;
   p.scale = a.scale;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.ld_dq = static_cast<int>(a.ld_dq);
@@ -573,6 +574,7 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
       }
     }
     p.kv_splits = splits;
+    p.wait_at_exit = 1;  // follows dK/dV on the stream and reads nothing it writes
     dim3 grid(static_cast<unsigned>(p.n_tblk * splits), static_cast<unsigned>(gy), B);
     if (splits > 1)
       return launch_k_cluster(sqa::bwd_dq_kernel<D, GradT, true>, grid, dim3(sqa::kBwdThreads), smem, st, splits,

@@ -161,6 +161,7 @@ struct BwdParams {
   int win_l, win_r;             // band: t - win_l <= u <= t + win_r (both <= N)
   int longest_first;            // causal: hand out the longest tiles first over the whole grid
   int kv_splits;                // dK/dV: CTAs (a cluster) sharing one key tile's steps; 1 = none
+  int wait_at_exit;             // dQ launched right after dK/dV: wait for that grid only before exiting
   float scale;
   float scale_log2;
 };
@@ -760,7 +761,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // the barrier, once this CTA holds its TMEM: a dependent CTA that took the
   // SM's columns first would wait for this grid while this CTA waited for
   // the columns.
-  grid_dependency_wait();
+  // Launched right after dK/dV (wait_at_exit), this grid reads nothing that
+  // grid writes: the inputs and the preprocess's statistics are complete
+  // once it may start (every dK/dV CTA releases its dependents only after
+  // its own wait on the preprocess has returned), so the work need not wait
+  // for dK/dV.  The wait moves to the exit, so that a kernel after this one
+  // on the stream still finds dK/dV complete.
+  if (!p.wait_at_exit) grid_dependency_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1009,6 +1016,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  if (p.wait_at_exit) grid_dependency_wait();
 }
 
 }  // namespace sqa
