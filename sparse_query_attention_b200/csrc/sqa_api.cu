@@ -684,15 +684,17 @@ sqa_status_t launch_gemm_pair(const CUtensorMap& ma, const CUtensorMap& mb, cons
 }
 
 // Split K over clusters (proj_gemm_splitk_kernel): for products with few
-// output tiles and a long K.  Clusters of 8, 4 or 2 CTAs, the largest for
-// which one cluster per output tile fits on the device at once and each CTA
-// keeps at least four K blocks; 0 when none does.
+// output tiles and a long K.  Clusters of 16 (a non-portable size, allowed
+// where the device runs it), 8, 4 or 2 CTAs: the largest for which one
+// cluster per output tile fits on the device at once and each CTA keeps at
+// least four K blocks; 0 when none does.
 template <int BN, bool kBf16, bool kAMN, bool kBMN>
 int gemm_split_count(long long tiles, int num_kb) {
   auto kern = sqa::proj_gemm_splitk_kernel<BN, kBf16, kAMN, kBMN>;
   constexpr int smem = sqa::SplitSmem<BN>::kDynamicBytes;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 0;
-  for (int splits = 8; splits >= 2; splits /= 2) {
+  const bool wide = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+  for (int splits = wide ? 16 : 8; splits >= 2; splits /= 2) {
     if (num_kb < 4 * splits) continue;
     if (tiles <= max_active_clusters(reinterpret_cast<const void*>(kern), splits, sqa::kProjThreads, smem))
       return splits;
