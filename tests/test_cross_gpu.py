@@ -179,3 +179,9 @@ def test_cross_forward_split_key_range(sqa, B, N_q, N_kv, H_q, H_kv, odt):
     assert_close(f64(o1), ro, "O")
     assert_close(f64(l1), rl, "LSE")
     assert torch.equal(o1, o2) and torch.equal(l1, l2), "forward differs between two runs"
+    # Without the LSE output the merged O is the same.
+    o3 = torch.empty_like(o1)
+    dt = sqa.SQA_DT_BF16 if odt == torch.bfloat16 else sqa.SQA_DT_F32
+    sqa.sqa_attn_fwd_cross(x["q"], x["k"], x["v"], o3, dt, None, B, N_q, N_kv, H_q, H_kv, d, 1 / math.sqrt(d))
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o3), "O differs without the LSE output"

@@ -29,6 +29,11 @@ def sqa():
     (2, 300, 8, 8, 128, False),
     (1, 513, 4, 1, 16, True),
     (3, 129, 6, 2, 64, False),
+    # Non-causal with few key tiles / query tiles: dK/dV split over clusters
+    # (d = 64), and the forward, dK/dV and dQ splits (d = 128), all writing
+    # through the packed strides.
+    (1, 2048, 8, 4, 64, False),
+    (1, 2048, 4, 4, 128, False),
 ])
 def test_packed_matches_oracle_and_dense(sqa, B, N, H_q, H_kv, d, causal):
     x = attention_inputs(B, N, H_q, H_kv, d, seed=400 + N, with_dout=True, device="cuda")
