@@ -18,13 +18,18 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  *  - All tensor pointers are DEVICE pointers owned by the caller.  The
- *    library allocates no device memory and keeps no per-call state.
+ *    library allocates no device memory and keeps no per-call state; on the
+ *    host it caches driver entry points and, per device, kernel and cluster
+ *    size, how many thread-block clusters run at once (queried once).
  *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
  *    NULL means the legacy default stream).  Nothing synchronises except
  *    sqa_device_status().  Kernels are launched as programmatic dependents
  *    of the previous kernel on the stream: they may start their set-up
- *    while it finishes but touch no global memory before it has completed,
- *    so stream order holds for every buffer, as with ordinary launches.
+ *    while it finishes but touch no global memory before the kernels of
+ *    earlier calls have completed, so stream order holds for every buffer,
+ *    as with ordinary launches.  (Inside one call, a kernel that reads
+ *    nothing its predecessor writes, dQ after dK/dV, starts its work early
+ *    and waits for that predecessor before it exits.)
  *  - Layouts are dense, row-major, with the last index contiguous:
  *      Q, O, dO, dQ : [B, N, H_q,  d_head]
  *      K, V, dK, dV : [B, N, H_kv, d_head]
