@@ -28,8 +28,9 @@
  *    while it finishes but touch no global memory before the kernels of
  *    earlier calls have completed, so stream order holds for every buffer,
  *    as with ordinary launches.  (Inside one call, a kernel that reads
- *    nothing its predecessor writes, dQ after dK/dV, starts its work early
- *    and waits for that predecessor before it exits.)
+ *    nothing its predecessor writes, dQ after dK/dV or the second of two
+ *    forward launches over one problem, starts its work early and waits
+ *    for that predecessor before it exits.)
  *  - Layouts are dense, row-major, with the last index contiguous:
  *      Q, O, dO, dQ : [B, N, H_q,  d_head]
  *      K, V, dK, dV : [B, N, H_kv, d_head]
