@@ -603,6 +603,15 @@ def time_projection(sqa, torch, stream, dev, reps=10):
             "cublas_ms": ms_r, "cublas_tflops": flops / ms_r / 1e9}
 
 
+def secondary_leg(fn):
+    """Runs one secondary measurement; an exception becomes {"error": ...}
+    in the JSON line instead of ending the run."""
+    try:
+        return fn()
+    except Exception as e:  # noqa: BLE001 - any failure is reported, none is hidden
+        return {"error": f"{type(e).__name__}: {e}"[:400]}
+
+
 def load_hbm_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -942,13 +951,16 @@ def run_sqa(args):
         variants[name]["speedup_vs_mha"] = variants["MHA"]["ms"] / variants[name]["ms"]
         variants[name]["ideal_speedup"] = VARIANTS["MHA"][0] / variants[name]["H_q"]
     sqa.sqa_device_status(stream)
-    training = time_training_step(sqa, torch, stream, flush, dev)
-    layer = time_decoder_layer(sqa, torch, stream, flush, dev)
-    long_seq = time_long_sequences(sqa, torch, stream, dev)
-    windowed = time_windowed(sqa, torch, stream, dev)
-    decode = time_decode(sqa, torch, stream, dev)
-    cross = time_cross(sqa, torch, stream, dev)
-    projection = time_projection(sqa, torch, stream, dev)
+    # The secondary legs (no collectives): a failure in one is recorded in
+    # its place in the line instead of ending the run, so the measurement
+    # above is still reported.
+    training = secondary_leg(lambda: time_training_step(sqa, torch, stream, flush, dev))
+    layer = secondary_leg(lambda: time_decoder_layer(sqa, torch, stream, flush, dev))
+    long_seq = secondary_leg(lambda: time_long_sequences(sqa, torch, stream, dev))
+    windowed = secondary_leg(lambda: time_windowed(sqa, torch, stream, dev))
+    decode = secondary_leg(lambda: time_decode(sqa, torch, stream, dev))
+    cross = secondary_leg(lambda: time_cross(sqa, torch, stream, dev))
+    projection = secondary_leg(lambda: time_projection(sqa, torch, stream, dev))
 
     peak, peak_kind = load_peaks()
     achieved = flops_step / (statistics.mean(per_launch_ms) / 1e3) / 1e12
@@ -981,7 +993,7 @@ def run_sqa(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = {k: v for k, v in cpu_baseline().items() if k not in ("seconds",)}
-        line["cpu_baseline"]["configs"] = cpu_baseline_configs()
+        line["cpu_baseline"]["configs"] = secondary_leg(cpu_baseline_configs)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
