@@ -31,7 +31,7 @@ def _nvcc() -> str:
 def _sources():
     out = [os.path.join(INCLUDE, "sqa.h")]
     for name in sorted(os.listdir(CSRC)):
-        if name.endswith((".cu", ".cuh")):
+        if name.endswith((".cu", ".cuh", ".h")):
             out.append(os.path.join(CSRC, name))
     return out
 

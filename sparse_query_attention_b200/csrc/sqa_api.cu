@@ -16,12 +16,18 @@
 #include "sqa_fwd_kernel.cuh"
 #include "sqa_fwd_quad_kernel.cuh"
 #include "sqa_fwd_split_kernel.cuh"
+#include "sqa_plan.h"
 #include "sqa_proj_kernel.cuh"
 #include "sqa_ptx.cuh"
 
 namespace {
 
 using sqa::kProjBM;
+using sqa::plan::cluster_split;
+using sqa::plan::decode_plan;
+using sqa::plan::DecodePlan;
+using sqa::plan::gemm_group_m;
+using sqa::plan::head_pack;
 
 // ---------------------------------------------------------------------------
 // Driver entry point for cuTensorMapEncodeTiled, fetched once through the
@@ -253,12 +259,6 @@ CUtensorMapSwizzle tma_swizzle_for_row_bytes(int row_bytes) {
                           : (row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
 }
 
-// Packing factor: the largest power of two dividing G, at most 128.
-int head_pack(int G) {
-  int g = 1;
-  while (g < 128 && (G % (2 * g)) == 0) g *= 2;
-  return g;
-}
 
 template <int D>
 sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* out, int out_bf16, float* lse,
@@ -318,17 +318,8 @@ sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* ou
       return SQA_ERR_CUDA;
     return launch_k(kern, grid, dim3(sqa::kQuadThreads), sqa::QuadCfg<D>::kSmemBytes, st, mq, mk, mv, p);
   } else {
-    // Three ways to cover an unmasked problem's query tiles, chosen by their
-    // wave counts on this GPU's SMs (one CTA per SM): the two-tile grid (two
-    // query tiles per CTA); the split grid (one tile per CTA, its two
-    // softmax tiles on the even and odd key blocks, so half the work per CTA
-    // at a rate measured ~8 % lower: a split wave costs kSplitWave of a
-    // two-tile wave); or both, the two-tile kernel on the token blocks that
-    // fill whole waves and the split kernel on the remaining tiles, launched
-    // after it on the stream (its CTAs start on the SMs the last two-tile
-    // wave frees, and wait for that grid only before exiting).  Under a band mask the work per CTA varies and the
-    // longest-first order already packs the waves (causal B=4, N=8192, (8,4)
-    // ran 2 % slower split), so masked problems keep the two-tile grid.
+    // The cover of the query tiles (two-tile grid, split grid, or both) is
+    // sqa::plan::fwd_wave_plan (sqa_plan.h), after the key-range split below.
     const int sms = num_sms();
     if (sms <= 0) return SQA_ERR_CUDA;
     // Few query tiles against many keys (unmasked: cross attention from a
@@ -343,32 +334,17 @@ sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* ou
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
         return SQA_ERR_CUDA;
       const long long units = static_cast<long long>(p.n_tblk) * gy * B;
-      const int nb = (Nkv + 127) / 128;
-      int splits = 1;
-      for (int c = 2; c <= 8; c *= 2) {
-        if (nb < 4 * c) break;
-        if (units > max_active_clusters(reinterpret_cast<const void*>(kern), c, sqa::kFwdThreads, C::kSmemBytes))
-          break;
-        splits = c;
-      }
+      const int splits = cluster_split(units, (Nkv + 127) / 128, 4, 8, [&](int c) {
+        return max_active_clusters(reinterpret_cast<const void*>(kern), c, sqa::kFwdThreads, C::kSmemBytes);
+      });
       if (splits > 1) {
         p.kv_splits = splits;
         const dim3 grid_c(static_cast<unsigned>(p.n_tblk * splits), static_cast<unsigned>(gy), B);
         return launch_k_cluster(kern, grid_c, dim3(sqa::kFwdThreads), C::kSmemBytes, st, splits, mq, mk, mv, p);
       }
     }
-    constexpr double kSplitWave = 0.55;
-    const long long yz = gy * B;
     const int n_tiles = (N + T - 1) / T;
-    auto waves = [&](long long ctas) { return static_cast<double>((ctas + sms - 1) / sms); };
-    const double t_two = waves(static_cast<long long>(p.n_tblk) * yz);
-    const double t_split = kSplitWave * waves(static_cast<long long>(n_tiles) * yz);
-    // mixed: the largest number of token blocks whose two-tile CTAs fill whole waves
-    const int n_a = static_cast<int>((static_cast<long long>(p.n_tblk) * yz / sms) * sms / yz);
-    const double t_mix = n_a > 0 && n_a < p.n_tblk
-                             ? waves(static_cast<long long>(n_a) * yz) +
-                                   kSplitWave * waves(static_cast<long long>(n_tiles - 2 * n_a) * yz)
-                             : 1e30;
+    const sqa::plan::FwdWavePlan cover = sqa::plan::fwd_wave_plan(p.n_tblk, gy * B, n_tiles, sms, a.masked);
     auto launch_split = [&](int tile0, int tiles) -> sqa_status_t {
       sqa::FwdParams ps = p;
       ps.n_tblk = n_tiles;
@@ -381,15 +357,15 @@ sqa_status_t launch_fwd_tc(const void* q, const void* k, const void* v, void* ou
         return SQA_ERR_CUDA;
       return launch_k(kern, grid1, dim3(sqa::kFwdThreads), smem, st, mq, mk, mv, ps);
     };
-    if (!a.masked && t_split < 0.97 * t_two && t_split <= t_mix) return launch_split(0, n_tiles);
-    if (!a.masked && t_mix < 0.97 * t_two) {
+    if (cover.cover == sqa::plan::FwdCover::kSplit) return launch_split(0, n_tiles);
+    if (cover.cover == sqa::plan::FwdCover::kMixed) {
       auto kern = sqa::sqa_fwd_kernel<D>;
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
         return SQA_ERR_CUDA;
-      dim3 grid_a(n_a, static_cast<unsigned>(gy), B);
+      dim3 grid_a(cover.n_a, static_cast<unsigned>(gy), B);
       const sqa_status_t s2 = launch_k(kern, grid_a, dim3(sqa::kFwdThreads), C::kSmemBytes, st, mq, mk, mv, p);
       if (s2 != SQA_OK) return s2;
-      return launch_split(2 * n_a, n_tiles - 2 * n_a);
+      return launch_split(2 * cover.n_a, n_tiles - 2 * cover.n_a);
     }
     auto kern = sqa::sqa_fwd_kernel<D>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
@@ -537,11 +513,9 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
       auto kern_s = sqa::bwd_dkdv_kernel<D, GradT, true, true>;
       if (cudaFuncSetAttribute(kern_s, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return SQA_ERR_CUDA;
-      for (int c = 2; c <= 8; c *= 2) {
-        if (n_all < 8LL * c) break;
-        if (units > max_active_clusters(reinterpret_cast<const void*>(kern_s), c, sqa::kBwdThreads, smem)) break;
-        splits = c;
-      }
+      splits = cluster_split(units, n_all, 8, 8, [&](int c) {
+        return max_active_clusters(reinterpret_cast<const void*>(kern_s), c, sqa::kBwdThreads, smem);
+      });
     }
     p.kv_splits = splits;
     dim3 grid(static_cast<unsigned>(((Nkv + 127) / 128) * splits), H_kv, B);
@@ -567,11 +541,9 @@ sqa_status_t launch_bwd_tc(const void* q, const void* k, const void* v, const vo
         return SQA_ERR_CUDA;
       const long long units = static_cast<long long>(p.n_tblk) * gy * B;
       const long long n_all = (Nkv + 63) / 64;
-      for (int c = 2; c <= 8; c *= 2) {
-        if (n_all < 8LL * c) break;
-        if (units > max_active_clusters(reinterpret_cast<const void*>(kern_s), c, sqa::kBwdThreads, smem)) break;
-        splits = c;
-      }
+      splits = cluster_split(units, n_all, 8, 8, [&](int c) {
+        return max_active_clusters(reinterpret_cast<const void*>(kern_s), c, sqa::kBwdThreads, smem);
+      });
     }
     p.kv_splits = splits;
     p.wait_at_exit = 1;  // follows dK/dV on the stream and reads nothing it writes
@@ -618,18 +590,6 @@ sqa_status_t attn_bwd_impl(const void* q, const void* k, const void* v, const vo
 // ---------------------------------------------------------------------------
 // Projection GEMM
 // ---------------------------------------------------------------------------
-// Raster of the persistent GEMMs (row tiles per group of the tile walk):
-// the smaller operand stays resident in L2 while the other streams through
-// once.  kResident leaves most of the 126 MB L2 (two halves, one per die) to
-// the streamed operand's tiles in flight and to the output.
-int gemm_group_m(int M, int N, int K, int bm) {
-  constexpr long long kResident = 40ll << 20;
-  const long long a_bytes = 2ll * M * K;
-  const long long b_bytes = 2ll * N * K;
-  if (b_bytes <= kResident && b_bytes <= a_bytes) return 1;  // N fastest: B stays
-  if (a_bytes <= kResident) return (M + bm - 1) / bm;        // M fastest: A stays
-  return 8;  // both large: groups of 8 row tiles share each pass over B
-}
 
 template <int BN, bool kBf16, bool kAMN, bool kBMN>
 sqa_status_t launch_gemm_bn(const CUtensorMap& ma, const CUtensorMap& mb, const float* bias, void* c, int M, int N,
@@ -694,12 +654,10 @@ int gemm_split_count(long long tiles, int num_kb) {
   constexpr int smem = sqa::SplitSmem<BN>::kDynamicBytes;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 0;
   const bool wide = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
-  for (int splits = wide ? 16 : 8; splits >= 2; splits /= 2) {
-    if (num_kb < 4 * splits) continue;
-    if (tiles <= max_active_clusters(reinterpret_cast<const void*>(kern), splits, sqa::kProjThreads, smem))
-      return splits;
-  }
-  return 0;
+  const int splits = cluster_split(tiles, num_kb, 4, wide ? 16 : 8, [&](int c) {
+    return max_active_clusters(reinterpret_cast<const void*>(kern), c, sqa::kProjThreads, smem);
+  });
+  return splits > 1 ? splits : 0;
 }
 
 template <int BN, bool kBf16, bool kAMN, bool kBMN>
@@ -854,51 +812,7 @@ sqa_status_t gemm_impl(const void* a, bool a_mn, const void* b, bool b_mn, const
 // ---------------------------------------------------------------------------
 // KV-cache decode
 // ---------------------------------------------------------------------------
-// Chunking of the cache: at least two waves of two CTAs per SM over the
-// (batch, key/value head, head sub-group) units, chunks of at least 256
-// keys and a multiple of the 64-key step; among split counts up to four
-// times that minimum, the smallest whose last wave is at least 95 % full
-// (else the fullest).  Fewer, longer chunks (one wave at most) measured
-// 1-6 % faster on a cool GPU but 2-25 % slower after seconds of tensor work
-// at the power cap.  Depends only on the shape, so the workspace size is
-// known before the lengths are.
-constexpr int kNumSMs = 148;
-constexpr int kDecodeSlots = 2 * kNumSMs;  // CTAs resident at once
-
-struct DecodePlan {
-  int g, log2g, n_sub, chunk, n_split;
-};
-
-DecodePlan decode_plan(int B, int H_q, int H_kv, int L_max) {
-  DecodePlan pl;
-  const int G = H_q / H_kv;
-  pl.g = head_pack(G);
-  pl.log2g = 0;
-  while ((1 << pl.log2g) < pl.g) ++pl.log2g;
-  pl.n_sub = G / pl.g;
-  const long long units = static_cast<long long>(B) * H_kv * pl.n_sub;
-  const long long max_split = (L_max + 255) / 256 > 0 ? (L_max + 255) / 256 : 1;
-  const long long n_min = std::min(max_split, std::max(1LL, (2LL * kDecodeSlots + units - 1) / units));
-  const long long n_max = std::min(max_split, 4 * n_min);
-  long long n = n_min;
-  double best = -1.0;
-  for (long long c = n_min; c <= n_max; ++c) {
-    const long long ctas = units * c;
-    const double fill = static_cast<double>(ctas) / (((ctas + kDecodeSlots - 1) / kDecodeSlots) * kDecodeSlots);
-    if (fill >= 0.95) {
-      n = c;
-      break;
-    }
-    if (fill > best) {
-      best = fill;
-      n = c;
-    }
-  }
-  const long long per = (L_max + n - 1) / n;
-  pl.chunk = static_cast<int>((per + 63) / 64 * 64);
-  pl.n_split = static_cast<int>((L_max + pl.chunk - 1) / pl.chunk);
-  return pl;
-}
+// Chunking of the cache: sqa::plan::decode_plan (sqa_plan.h).
 
 size_t decode_part_l_bytes(int n_split, int B, int n_new, int H_q) {
   const size_t n = static_cast<size_t>(n_split) * B * n_new * H_q * sizeof(float);
